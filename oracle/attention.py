@@ -1,0 +1,101 @@
+"""Bidirectional joint text+image attention with rotary Q/K, in fp64.
+
+What is computed, for every batch item b and head h separately (the heads of
+a DiT block attend independently; text and image tokens of one item form one
+sequence that every token attends to in full, which is the "shared attention
+layer" of bpdata.com "FLUX 3 Image Klein optimalizálása", section
+"Modellezés és pipeline jellemzők"):
+
+    q~_n = R(pos_n) q_n,   k~_m = R(pos_m) k_m          (oracle.rope)
+    s_nm = (q~_n . k~_m) * scale,   scale = 1 / sqrt(D)
+    O_n  = sum_m softmax_m(s_n.) v_m
+    LSE_n = log sum_m exp(s_nm)          (natural log, scaled-logit units)
+
+written as the definition: a full row of logits, its maximum subtracted
+before exp (which changes nothing mathematically), the exponentials summed,
+and one weighted sum of V.  No tiling, streaming or rescaling.
+
+`round_rotated="bf16"` rounds q~ and k~ to the nearest bf16 after the exact
+rotation: the operand precision of a bf16 tensor-core product of rotated
+tiles.  Everything else stays fp64.
+
+Test infrastructure only (see oracle/__init__.py).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import formats, rope
+
+
+def to_f64(x) -> np.ndarray:
+    """Exact fp64 copy of a numpy array or a (CPU) torch tensor of any float dtype."""
+    if hasattr(x, "detach"):
+        import torch
+        return x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def attention_rows(q_rows, k, v, scale):
+    """softmax(q_rows k^T * scale) v for one (b, h): returns O [R, D], LSE [R]."""
+    s = (q_rows @ k.T) * scale
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    out = (e @ v) / l
+    lse = m[:, 0] + np.log(l[:, 0])
+    return out, lse
+
+
+def probabilities(q_rows, k, scale):
+    """Full attention probability rows softmax(q_rows k^T * scale) [R, N]."""
+    s = (q_rows @ k.T) * scale
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def _round(x, how):
+    if how is None:
+        return x
+    if how == "bf16":
+        return formats.round_bf16(x)
+    if how == "fp16":
+        return formats.round_fp16(x)
+    raise ValueError(how)
+
+
+def joint_attention(q, k, v, pos=None, rows=None, axes=rope.DEFAULT_AXES,
+                    theta: float = rope.DEFAULT_THETA, scale=None, round_rotated=None):
+    """Oracle output for tensors q, k, v [B, H, N, D].
+
+    pos:  int [N, 3] token positions (t, h, w) or None for no rotary embedding.
+    rows: int [R, 3] (b, h, n) query rows to evaluate, or None for all rows.
+    Returns (O [R, D], LSE [R]) in fp64, in the order of `rows` (row-major
+    (b, h, n) order when rows is None).
+    """
+    B, H, N, D = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    if rows is None:
+        b, h, n = np.meshgrid(np.arange(B), np.arange(H), np.arange(N), indexing="ij")
+        rows = np.stack([b.reshape(-1), h.reshape(-1), n.reshape(-1)], axis=1)
+    rows = np.asarray(rows, dtype=np.int64)
+    phi = rope.angles(pos, axes, theta) if pos is not None else None
+    out = np.empty((len(rows), D), dtype=np.float64)
+    lse = np.empty(len(rows), dtype=np.float64)
+    keys = rows[:, 0] * (H + 1) + rows[:, 1]
+    for key in np.unique(keys):
+        idx = np.nonzero(keys == key)[0]
+        bb, hh = int(rows[idx[0], 0]), int(rows[idx[0], 1])
+        kk = to_f64(k[bb, hh])
+        vv = to_f64(v[bb, hh])
+        qq = to_f64(q[bb, hh][rows[idx, 2]])
+        if phi is not None:
+            kk = rope.rotate(kk, phi)
+            qq = rope.rotate(qq, phi[rows[idx, 2]])
+        kk = _round(kk, round_rotated)
+        qq = _round(qq, round_rotated)
+        o, l = attention_rows(qq, kk, vv, scale)
+        out[idx] = o
+        lse[idx] = l
+    return out, lse
