@@ -1,0 +1,123 @@
+"""Python binding of libdit_attn, the B200 joint text+image attention library.
+
+Argument marshalling only: every function below hands raw device pointers,
+sizes and the stream to the C entry point of the same name (declared in
+include/dit_attn.h).  Torch tensors serve as device buffers; all computation
+happens in the library's CUDA kernels.  There is no fallback: if the shared
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+from ._lib import load_library, library_path  # noqa: F401
+
+DIT_OK = 0
+DIT_ERR_INVALID_ARG = -1
+DIT_ERR_UNSUPPORTED = -2
+DIT_ERR_MISALIGNED = -3
+DIT_ERR_CUDA = -4
+DIT_ERR_TIMEOUT = -5
+DIT_BF16 = 0
+DIT_FP8_E4M3 = 1
+DIT_OUT_F32 = 0x100
+
+
+class DitError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (what, dit_attn_status_string(status), status))
+
+
+def _check(status: int, what: str) -> None:
+    if status != DIT_OK:
+        raise DitError(status, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _require(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def dit_rope_table_build(pos, axes: Sequence[int], theta: float, rope_cos, rope_sin, stream=None) -> None:
+    """Fill rope_cos / rope_sin (CUDA fp32 [N, 64]) from positions pos (CUDA int32 [N, 3])."""
+    import torch
+    _require(pos.is_cuda and pos.dtype == torch.int32 and pos.dim() == 2 and pos.shape[1] == 3 and
+             pos.is_contiguous(), "pos must be a contiguous CUDA int32 [N, 3] tensor")
+    N = pos.shape[0]
+    for t in (rope_cos, rope_sin):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (N, 64),
+                 "rope tables must be contiguous CUDA fp32 [N, 64] tensors")
+    ax = (ctypes.c_int32 * 3)(*[int(a) for a in axes])
+    _check(load_library().dit_rope_table_build(_ptr(pos), N, 128, ax, float(theta), _ptr(rope_cos),
+                                               _ptr(rope_sin), _stream(stream)), "dit_rope_table_build")
+
+
+def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: int, dtype: int = DIT_BF16,
+                     stream=None) -> None:
+    """out (and lse, if not None) <- joint attention of bf16 q, k, v [B, H, N, D] on the GPU."""
+    import torch
+    _require(q.dim() == 4 and q.shape == k.shape == v.shape, "q, k, v must share one [B, H, N, D] shape")
+    B, H, N, D = q.shape
+    _require(N == n_txt + n_img, "N must equal n_txt + n_img")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "q, k, v must be contiguous CUDA bf16")
+    out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
+    _require(out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q.shape,
+             "out must be a contiguous CUDA tensor of q's shape and the requested dtype")
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, N),
+                 "lse must be a contiguous CUDA fp32 [B, H, N] tensor")
+    if rope_cos is not None or rope_sin is not None:
+        for t in (rope_cos, rope_sin):
+            _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _check(load_library().dit_attn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(out),
+                                           _ptr(lse), B, H, n_txt, n_img, D, dtype, _stream(stream)),
+           "dit_attn_forward")
+
+
+def dit_attn_get_status(stream=None) -> int:
+    """Synchronise the stream, return and clear the device status word."""
+    st = ctypes.c_int(0)
+    _check(load_library().dit_attn_get_status(ctypes.byref(st), _stream(stream)), "dit_attn_get_status")
+    return st.value
+
+
+def dit_attn_status_string(status: int) -> str:
+    return load_library().dit_attn_status_string(int(status)).decode()
+
+
+# ----------------------------------------------------------- allocating helpers
+def rope_table(pos, axes=(16, 56, 56), theta: float = 10000.0, stream=None):
+    """Allocate and fill (cos, sin) tables for CUDA int32 positions [N, 3]."""
+    import torch
+    N = pos.shape[0]
+    c = torch.empty((N, 64), dtype=torch.float32, device=pos.device)
+    s = torch.empty_like(c)
+    dit_rope_table_build(pos, axes, theta, c, s, stream)
+    return c, s
+
+
+def forward(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool = False, with_lse: bool = True,
+            stream=None):
+    """Allocate out (and lse) and run dit_attn_forward; returns (out, lse)."""
+    import torch
+    B, H, N, D = q.shape
+    out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
+    dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt,
+                     DIT_BF16 | (DIT_OUT_F32 if out_f32 else 0), stream)
+    return out, lse

@@ -1,0 +1,113 @@
+// C-ABI entry points of libdit_attn: argument validation, status word and
+// dispatch to the kernel launchers.  Declarations and contracts live in
+// include/dit_attn.h.
+#include <cstdint>
+#include <mutex>
+
+#include "dit_attn.h"
+#include "launch.h"
+
+namespace dit {
+
+// The one static device allocation of the library: a status word that
+// kernels set when a bounded wait gives up.  Its device address differs per
+// device, so it is looked up with that device current and cached.
+__device__ int g_status_word = 0;
+
+int* device_status_word() {
+  constexpr int kMaxDevices = 64;
+  static int* cached[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<int*>(ptr);
+  }
+  return cached[dev];
+}
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace dit
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int dit_rope_table_build(const int32_t* pos, int N, int D, const int32_t* axes, double theta, float* rope_cos,
+                         float* rope_sin, dit_stream_t stream) {
+  if (pos == nullptr || axes == nullptr || rope_cos == nullptr || rope_sin == nullptr) return DIT_ERR_INVALID_ARG;
+  if (N < 1 || !(theta > 0.0)) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if (axes[0] < 0 || axes[1] < 0 || axes[2] < 0 || (axes[0] | axes[1] | axes[2]) & 1 ||
+      axes[0] + axes[1] + axes[2] != D)
+    return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(N) * (D / 2) > (1LL << 40)) return DIT_ERR_INVALID_ARG;
+  if (!aligned4(pos) || !aligned16(rope_cos) || !aligned16(rope_sin)) return DIT_ERR_MISALIGNED;
+  dit::RopeTableArgs a{pos, N, D, {axes[0], axes[1], axes[2]}, theta, rope_cos, rope_sin};
+  return dit::launch_rope_table(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                     void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                     dit_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N_txt < 0 || N_img < 0) return DIT_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img;
+  if (N < 1 || N > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if ((dtype & ~DIT_OUT_F32) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIT_ERR_MISALIGNED;
+  if ((rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) || (lse != nullptr && !aligned4(lse)))
+    return DIT_ERR_MISALIGNED;
+  dit::AttnFwdArgs a{q, k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N), (dtype & DIT_OUT_F32) != 0};
+  return dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream));
+}
+
+int dit_attn_get_status(int* status_host, dit_stream_t stream) {
+  if (status_host == nullptr) return DIT_ERR_INVALID_ARG;
+  int* word = dit::device_status_word();
+  if (word == nullptr) return DIT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int value = 0;
+  if (cudaMemcpyAsync(&value, word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return DIT_ERR_CUDA;
+  if (cudaMemsetAsync(word, 0, sizeof(int), s) != cudaSuccess) return DIT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DIT_ERR_CUDA;
+  *status_host = value;
+  return DIT_OK;
+}
+
+const char* dit_attn_status_string(int status) {
+  switch (status) {
+    case DIT_OK: return "ok";
+    case DIT_ERR_INVALID_ARG: return "invalid argument";
+    case DIT_ERR_UNSUPPORTED: return "unsupported head dimension, dtype or flag";
+    case DIT_ERR_MISALIGNED: return "pointer not aligned (16 bytes; 4 for lse)";
+    case DIT_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case DIT_ERR_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

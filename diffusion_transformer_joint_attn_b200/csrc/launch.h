@@ -1,0 +1,46 @@
+// Host-side launchers shared between the C-ABI shim and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace dit {
+
+// Device status word of the current device (see capi.cu).
+int* device_status_word();
+
+struct RopeTableArgs {
+  const int32_t* pos;
+  int N;
+  int D;
+  int axes[3];
+  double theta;
+  float* cos;
+  float* sin;
+};
+cudaError_t launch_rope_table(const RopeTableArgs& a, cudaStream_t s);
+
+struct AttnFwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* cos;
+  const float* sin;
+  void* out;
+  float* lse;
+  int B, H, N;
+  bool out_f32;
+};
+// Builds the tensor maps and launches the BF16 forward kernel.
+// Returns 0 on success, a negative dit_status_t otherwise.
+int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s);
+
+// cuTensorMapEncodeTiled, resolved once through the runtime's driver entry
+// point (no link-time dependency on libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+}  // namespace dit

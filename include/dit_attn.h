@@ -1,0 +1,126 @@
+/*
+ * dit_attn.h — C ABI of libdit_attn: joint text+image attention for
+ * FLUX-style diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Inside every DiT block the text tokens, the noisy
+ * target-image tokens and (for image-to-image) the reference-image tokens are
+ * concatenated and attend to each other in one shared, bidirectional attention
+ * layer (bpdata.com "FLUX 3 Image Klein optimalizálása", section "Modellezés
+ * és pipeline jellemzők").  Plain BF16 attention is about 60 % of the DiT's
+ * GPU kernel time at 2048x2048 (scopeai.cc FLUX 3 Klein story, section on the
+ * effect of each optimisation).  For each batch item b and head h:
+ *
+ *     q~_n = R(pos_n) q_n,  k~_m = R(pos_m) k_m      three-axis rotary embedding
+ *     O_n  = sum_m softmax_m(q~_n . k~_m / sqrt(D)) v_m
+ *     LSE_n = ln sum_m exp(q~_n . k~_m / sqrt(D))
+ *
+ * R(pos) turns channel pair (2j, 2j+1) by the angle pos_a * theta^(-2i/d_a),
+ * where axis a in (t, h, w) owns the consecutive channel slice of width d_a
+ * that contains the pair and i is the pair's index inside that slice.
+ *
+ * Conventions shared by every entry point:
+ *   - Layout: q, k, v, out are [B][H][N][D] row-major, N = N_txt + N_img
+ *     tokens in sequence order [text | image(s)]; lse is [B][H][N].
+ *   - Ownership: the caller allocates and owns every buffer.  The library
+ *     allocates no device memory per call; it keeps one static device status
+ *     word.  Inputs are only read; outputs are fully overwritten.
+ *   - Streams: every call is asynchronous on `stream` (a cudaStream_t, NULL =
+ *     legacy default stream) and does not synchronise the host, except
+ *     dit_attn_get_status.
+ *   - Errors: every call returns a dit_status_t.  Argument errors are found on
+ *     the host before anything is launched.  A device-side wait that exceeds
+ *     its time limit makes the kernel exit early and records DIT_ERR_TIMEOUT
+ *     in the status word, read by dit_attn_get_status.
+ */
+#ifndef DIT_ATTN_H
+#define DIT_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* dit_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  DIT_OK = 0,
+  DIT_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, sizes that overflow */
+  DIT_ERR_UNSUPPORTED = -2, /* D != 128, unknown dtype or flag */
+  DIT_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned (4-byte for lse) */
+  DIT_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+  DIT_ERR_TIMEOUT = -5      /* a device-side wait gave up (read via dit_attn_get_status) */
+} dit_status_t;
+
+/* Element type of q/k/v, OR-able with the flags below. */
+typedef enum { DIT_BF16 = 0, DIT_FP8_E4M3 = 1 } dit_dtype_t;
+#define DIT_OUT_F32 0x100 /* write `out` as fp32 instead of bf16 */
+
+/*
+ * dit_rope_table_build — cos/sin table of the three-axis rotary embedding.
+ *
+ *   pos       device int32 [N][3]: (t, h, w) position of every token.  In the
+ *             FLUX joint sequence text tokens sit at (0,0,0), target-image
+ *             latent pixel (row, col) at (0,row,col) and a reference image's at
+ *             (1,row,col).
+ *   N         number of tokens, >= 1.
+ *   D         head dimension, 128.
+ *   axes      HOST int32[3]: channels per axis (t, h, w), each even, sum == D,
+ *             e.g. {16, 56, 56}; slices are consecutive in that order.
+ *   theta     frequency base, > 0 (10000 for FLUX).
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2], written: entry [n][j] is cos/sin of the
+ *             angle of channel pair (2j, 2j+1) at token n,
+ *             pos[n][a] * theta^(-2i/d_a) with (a, i) the pair's axis and
+ *             index inside that axis; evaluated in fp64, rounded to fp32.
+ * Pointers 16-byte aligned.  Runs once per resolution, not per attention call.
+ */
+int dit_rope_table_build(const int32_t* pos, int N, int D, const int32_t* axes, double theta, float* rope_cos,
+                         float* rope_sin, dit_stream_t stream);
+
+/*
+ * dit_attn_forward — joint attention forward, BF16 in, BF16 (or fp32) out.
+ *
+ *   q, k, v   device bf16 [B][H][N][D], N = N_txt + N_img.
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2] from dit_rope_table_build, applied to q and
+ *             k inside the kernel; both NULL = no rotary embedding.
+ *   out       device [B][H][N][D], bf16, or fp32 when dtype has DIT_OUT_F32.
+ *   lse       device fp32 [B][H][N] or NULL: natural-log log-sum-exp of the
+ *             scaled logits q~.k~/sqrt(D) of every query row.
+ *   B, H      batch (e.g. 2 for the two classifier-free-guidance branches) and
+ *             heads, >= 1.
+ *   N_txt, N_img
+ *             text and image token counts, >= 0, N_txt + N_img >= 1.  Every
+ *             token attends to all N tokens (no mask); positions enter only
+ *             through the tables.
+ *   D         head dimension; must be 128.
+ *   dtype     DIT_BF16, optionally | DIT_OUT_F32.
+ *
+ * Precision: the rotation runs in fp32 and the rotated q, k are rounded to
+ * bf16 tensor-core operands; q~ k~^T accumulates in fp32; the softmax runs in
+ * fp32; P (in [0, 256]) and v are fp16 tensor-core operands (v must satisfy
+ * |v| <= 65504), P v accumulates in fp32.
+ * All pointers 16-byte aligned except lse (4-byte).  Graph-capturable: one
+ * kernel launch, no host synchronisation, no allocation.
+ */
+int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                     void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                     dit_stream_t stream);
+
+/*
+ * dit_attn_get_status — synchronise `stream`, copy the device status word to
+ * *status_host (DIT_OK or DIT_ERR_TIMEOUT) and reset it to DIT_OK.  Returns
+ * DIT_OK, or DIT_ERR_CUDA if the synchronisation or copy failed (for example
+ * after a device fault), or DIT_ERR_INVALID_ARG for a NULL status_host.
+ */
+int dit_attn_get_status(int* status_host, dit_stream_t stream);
+
+/* Static English description of a dit_status_t value. */
+const char* dit_attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_ATTN_H */

@@ -1,0 +1,56 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path on a workload and
+evaluate the fp64 oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import diffusion_transformer_joint_attn_b200 as dit
+import workloads as W
+from oracle import attention as oracle_attention
+
+# Parity bars of the BF16 path (max-abs / mean-abs over all checked output
+# elements; LSE in natural-log units of the scaled logits).
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+
+
+def lse_bound(lse_ref):
+    return 1e-3 + 1e-5 * np.abs(lse_ref)
+
+
+def device_inputs(w, seed=0):
+    q, k, v = W.make_qkv(w, seed)
+    return q, k, v, q.cuda(), k.cuda(), v.cuda()
+
+
+def rope_tables(w):
+    pos = torch.from_numpy(W.positions(w)).cuda()
+    return dit.rope_table(pos)
+
+
+def gather_rows(t, rows):
+    """t: [B, H, N, ...] tensor; rows: int [R, 3] (b, h, n) -> numpy [R, ...] fp64."""
+    idx = torch.from_numpy(rows).to(t.device)
+    return t[idx[:, 0], idx[:, 1], idx[:, 2]].double().cpu().numpy()
+
+
+def errors(got, ref):
+    e = np.abs(got - ref)
+    return float(e.max()), float(e.mean())
+
+
+def run_gpu(w, rope=True, out_f32=False, seed=0, inputs=None):
+    if inputs is None:
+        inputs = device_inputs(w, seed)
+    q, k, v, qd, kd, vd = inputs
+    cs = rope_tables(w) if rope else (None, None)
+    out, lse = dit.forward(qd, kd, vd, cs[0], cs[1], n_txt=w.n_txt, out_f32=out_f32)
+    torch.cuda.synchronize()
+    assert dit.dit_attn_get_status() == dit.DIT_OK
+    return out, lse
+
+
+def oracle_rows(w, q, k, v, rows, rope=True, round_rotated=None):
+    pos = W.positions(w) if rope else None
+    return oracle_attention.joint_attention(q, k, v, pos=pos, rows=rows, round_rotated=round_rotated)

@@ -1,0 +1,93 @@
+"""The C ABI: the library loads, exports every entry point include/dit_attn.h
+declares, and rejects bad arguments on the host before touching a GPU.  CPU only."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import diffusion_transformer_joint_attn_b200 as dit
+from diffusion_transformer_joint_attn_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(dit_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "dit_attn_forward" in names and "dit_rope_table_build" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    # the binding knows each of them too
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert dit.dit_attn_status_string(0) == "ok"
+    assert "timed out" in dit.dit_attn_status_string(-5)
+    assert dit.dit_attn_status_string(12345) == "unknown status"
+
+
+def _fwd(lib, q=0x10000, k=0x20000, v=0x30000, cos=None, sin=None, out=0x40000, lse=None, B=1, H=1, nt=8, ni=8, D=128,
+         dtype=0):
+    return lib.dit_attn_forward(q, k, v, cos, sin, out, lse, B, H, nt, ni, D, dtype, None)
+
+
+def test_forward_argument_errors(lib):
+    # every case below fails validation before any CUDA call
+    assert _fwd(lib, q=None) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, out=None) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, cos=0x50000) == dit.DIT_ERR_INVALID_ARG          # sin missing
+    assert _fwd(lib, B=0) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, H=-1) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, nt=0, ni=0) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, nt=-3) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, nt=2 ** 31 - 1, ni=2) == dit.DIT_ERR_INVALID_ARG
+    assert _fwd(lib, D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=dit.DIT_FP8_E4M3) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=0x400) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, q=0x10008) == dit.DIT_ERR_MISALIGNED
+    assert _fwd(lib, out=0x40004) == dit.DIT_ERR_MISALIGNED
+    assert _fwd(lib, cos=0x50000, sin=0x60008) == dit.DIT_ERR_MISALIGNED
+    assert _fwd(lib, lse=0x70002) == dit.DIT_ERR_MISALIGNED
+
+
+def test_rope_table_argument_errors(lib):
+    ax = (ctypes.c_int32 * 3)(16, 56, 56)
+    bad = (ctypes.c_int32 * 3)(16, 55, 57)
+    short = (ctypes.c_int32 * 3)(16, 56, 50)
+    f = lib.dit_rope_table_build
+    assert f(None, 8, 128, ax, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x100, 0, 128, ax, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x100, 8, 128, ax, 0.0, 0x1000, 0x2000, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x100, 8, 128, bad, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x100, 8, 128, short, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x100, 8, 96, ax, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_UNSUPPORTED
+    assert f(0x102, 8, 128, ax, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_MISALIGNED
+    assert f(0x100, 8, 128, ax, 1e4, 0x1004, 0x2000, None) == dit.DIT_ERR_MISALIGNED
+
+
+def test_get_status_rejects_null(lib):
+    assert lib.dit_attn_get_status(None, None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_binding_marshalling_errors():
+    import torch
+    q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dit.dit_attn_forward(q, q, q, None, None, q, None, 2, 2)      # CPU tensors are refused
