@@ -15,9 +15,13 @@ written as the definition: a full row of logits, its maximum subtracted
 before exp (which changes nothing mathematically), the exponentials summed,
 and one weighted sum of V.  No tiling, streaming or rescaling.
 
-`round_rotated="bf16"` rounds q~ and k~ to the nearest bf16 after the exact
-rotation: the operand precision of a bf16 tensor-core product of rotated
-tiles.  Everything else stays fp64.
+Two optional rounding points model the formats the library's interface fixes
+for intermediate values, with exact arithmetic in between:
+* `table_fp32=True` rotates with the cos / sin table entries rounded to fp32
+  (the table format the attention call takes);
+* `round_rotated="bf16"` rounds the exactly rotated q~ and k~ to the nearest
+  bf16 (ties to even): the operand precision of a bf16 tensor-core product.
+Everything else stays fp64.
 
 Test infrastructure only (see oracle/__init__.py).
 """
@@ -65,7 +69,7 @@ def _round(x, how):
 
 
 def joint_attention(q, k, v, pos=None, rows=None, axes=rope.DEFAULT_AXES,
-                    theta: float = rope.DEFAULT_THETA, scale=None, round_rotated=None):
+                    theta: float = rope.DEFAULT_THETA, scale=None, round_rotated=None, table_fp32=False):
     """Oracle output for tensors q, k, v [B, H, N, D].
 
     pos:  int [N, 3] token positions (t, h, w) or None for no rotary embedding.
@@ -80,7 +84,9 @@ def joint_attention(q, k, v, pos=None, rows=None, axes=rope.DEFAULT_AXES,
         b, h, n = np.meshgrid(np.arange(B), np.arange(H), np.arange(N), indexing="ij")
         rows = np.stack([b.reshape(-1), h.reshape(-1), n.reshape(-1)], axis=1)
     rows = np.asarray(rows, dtype=np.int64)
-    phi = rope.angles(pos, axes, theta) if pos is not None else None
+    cs = None
+    if pos is not None:
+        cs = rope.table_fp32(pos, axes, theta) if table_fp32 else rope.table(pos, axes, theta)
     out = np.empty((len(rows), D), dtype=np.float64)
     lse = np.empty(len(rows), dtype=np.float64)
     keys = rows[:, 0] * (H + 1) + rows[:, 1]
@@ -90,9 +96,9 @@ def joint_attention(q, k, v, pos=None, rows=None, axes=rope.DEFAULT_AXES,
         kk = to_f64(k[bb, hh])
         vv = to_f64(v[bb, hh])
         qq = to_f64(q[bb, hh][rows[idx, 2]])
-        if phi is not None:
-            kk = rope.rotate(kk, phi)
-            qq = rope.rotate(qq, phi[rows[idx, 2]])
+        if cs is not None:
+            kk = rope.rotate_with_table(kk, cs[0], cs[1])
+            qq = rope.rotate_with_table(qq, cs[0][rows[idx, 2]], cs[1][rows[idx, 2]])
         kk = _round(kk, round_rotated)
         qq = _round(qq, round_rotated)
         o, l = attention_rows(qq, kk, vv, scale)

@@ -50,11 +50,21 @@ def table(pos, axes=DEFAULT_AXES, theta: float = DEFAULT_THETA):
     return np.cos(phi), np.sin(phi)
 
 
+def table_fp32(pos, axes=DEFAULT_AXES, theta: float = DEFAULT_THETA):
+    """The table as the library stores it: each fp64 entry rounded to the
+    nearest fp32 value (returned as fp64)."""
+    c, s = table(pos, axes, theta)
+    return c.astype(np.float32).astype(np.float64), s.astype(np.float32).astype(np.float64)
+
+
 def rotate(x, phi):
     """Apply the rotation of angle table `phi` [N, D/2] to x [..., N, D] (fp64)."""
+    return rotate_with_table(x, np.cos(phi), np.sin(phi))
+
+
+def rotate_with_table(x, c, s):
+    """Apply the rotation whose cos / sin entries are c, s [N, D/2] to x [..., N, D] (fp64)."""
     x = np.asarray(x, dtype=np.float64)
-    c = np.cos(phi)
-    s = np.sin(phi)
     xe = x[..., 0::2]
     xo = x[..., 1::2]
     out = np.empty_like(x)

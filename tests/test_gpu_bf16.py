@@ -33,14 +33,15 @@ def built():
     dit.load_library()
 
 
-def check(out, lse, rows, O_ref, L_ref, label):
+def check(out, lse, rows, O_ref, L_ref, label, gate_lse=True):
     got = gather_rows(out, rows)
     mx, mean = errors(got, O_ref)
     dl = np.abs(gather_rows(lse, rows) - L_ref)
     print("%s: max-abs %.3e mean-abs %.3e max|dLSE| %.3e (%d rows)" % (label, mx, mean, dl.max(), len(rows)))
     assert mx <= BF16_MAX_ABS, label
     assert mean <= BF16_MEAN_ABS, label
-    assert np.all(dl <= lse_bound(L_ref)), label
+    if gate_lse:
+        assert np.all(dl <= lse_bound(L_ref)), label
 
 
 def test_rope_table_matches_oracle():
@@ -62,7 +63,9 @@ def test_parity_plain_workloads(name):
     rows = W.sample_rows(w)
     O_ref, L_ref = oracle_rows(w, q, k, v, rows)
     out, lse = run_gpu(w, inputs=inputs)
-    check(out, lse, rows, O_ref, L_ref, name + " bf16-out vs exact")
+    # the LSE moves by ~1e-3 with the bf16 rounding of the rotated operands:
+    # it is gated against the operand-rounded oracle below
+    check(out, lse, rows, O_ref, L_ref, name + " bf16-out vs exact", gate_lse=False)
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
     O_op, L_op = oracle_rows(w, q, k, v, rows, round_rotated="bf16")
     check(out32, lse32, rows, O_op, L_op, name + " fp32-out vs bf16-operand oracle")
@@ -103,7 +106,7 @@ def test_parity_ragged_shapes(B, H, n_txt, grids):
     rows = W.sample_rows(w)
     O_ref, L_ref = oracle_rows(w, q, k, v, rows)
     out, lse = run_gpu(w, inputs=inputs)
-    check(out, lse, rows, O_ref, L_ref, "ragged N=%d bf16-out" % w.N)
+    check(out, lse, rows, O_ref, L_ref, "ragged N=%d bf16-out" % w.N, gate_lse=False)
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
     O_op, L_op = oracle_rows(w, q, k, v, rows, round_rotated="bf16")
     check(out32, lse32, rows, O_op, L_op, "ragged N=%d fp32-out" % w.N)

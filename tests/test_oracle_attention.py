@@ -240,3 +240,21 @@ def test_sampled_rows_equal_the_same_rows_of_the_full_result():
     Os, Ls = attention.joint_attention(q, k, v, pos=pos, rows=rows)
     assert np.max(np.abs(Os - O[flat])) < 1e-13
     assert np.max(np.abs(Ls - L[flat])) < 1e-13
+
+
+def test_fp32_table_option_rounds_only_the_table():
+    rng = np.random.default_rng(14)
+    N, D = 40, 128
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    pos = rng.integers(0, 100, size=(N, 3))
+    c, s = rope.table(pos)
+    c32, s32 = rope.table_fp32(pos)
+    # nearest fp32: within half an fp32 ulp of the fp64 value, and on the fp32 grid
+    assert np.all(np.abs(c32 - c) <= 2.0 ** -25) and np.array_equal(c32, c32.astype(np.float32))
+    from oracle import formats
+    qr = formats.round_bf16(rope.rotate_with_table(q, c32, s32))
+    kr = formats.round_bf16(rope.rotate_with_table(k, c32, s32))
+    O_ref, L_ref = attention.attention_rows(qr, kr, v, 1 / math.sqrt(D))
+    O, L = attention.joint_attention(q[None, None], k[None, None], v[None, None], pos=pos, round_rotated="bf16",
+                                     table_fp32=True)
+    assert np.array_equal(O, O_ref) and np.array_equal(L, L_ref)
