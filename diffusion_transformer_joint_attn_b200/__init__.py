@@ -22,6 +22,7 @@ DIT_ERR_TIMEOUT = -5
 DIT_BF16 = 0
 DIT_FP8_E4M3 = 1
 DIT_OUT_F32 = 0x100
+DIT_K_ROTATED = 0x200
 
 
 class DitError(RuntimeError):
@@ -63,6 +64,20 @@ def dit_rope_table_build(pos, axes: Sequence[int], theta: float, rope_cos, rope_
     ax = (ctypes.c_int32 * 3)(*[int(a) for a in axes])
     _check(load_library().dit_rope_table_build(_ptr(pos), N, 128, ax, float(theta), _ptr(rope_cos),
                                                _ptr(rope_sin), _stream(stream)), "dit_rope_table_build")
+
+
+def dit_rope_apply(x, rope_cos, rope_sin, x_rot, stream=None) -> None:
+    """x_rot <- rotary embedding of bf16 x [B, H, N, D] (x_rot may be x)."""
+    import torch
+    _require(x.dim() == 4 and x.shape == x_rot.shape, "x and x_rot must share one [B, H, N, D] shape")
+    B, H, N, D = x.shape
+    for t in (x, x_rot):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "x, x_rot must be contiguous CUDA bf16")
+    for t in (rope_cos, rope_sin):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (N, D // 2),
+                 "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _check(load_library().dit_rope_apply(_ptr(x), _ptr(rope_cos), _ptr(rope_sin), _ptr(x_rot), B, H, N, D,
+                                         _stream(stream)), "dit_rope_apply")
 
 
 def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: int, dtype: int = DIT_BF16,
@@ -112,12 +127,12 @@ def rope_table(pos, axes=(16, 56, 56), theta: float = 10000.0, stream=None):
 
 
 def forward(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool = False, with_lse: bool = True,
-            stream=None):
+            k_rotated: bool = False, stream=None):
     """Allocate out (and lse) and run dit_attn_forward; returns (out, lse)."""
     import torch
     B, H, N, D = q.shape
     out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
-    dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt,
-                     DIT_BF16 | (DIT_OUT_F32 if out_f32 else 0), stream)
+    flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0)
+    dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt, DIT_BF16 | flags, stream)
     return out, lse

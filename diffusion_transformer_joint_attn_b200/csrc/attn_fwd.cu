@@ -20,6 +20,7 @@
 
 #include "launch.h"
 #include "ptx.cuh"
+#include "rope_exact.cuh"
 
 namespace dit {
 namespace {
@@ -59,6 +60,7 @@ struct Params {
   int n_kv;
   int pairs;          // query-tile pairs per (b, h)
   int out_f32;
+  int rotate_k;       // rotate K tiles in the kernel (0: K arrives rotated or no rotary embedding)
   float scale_log2;   // log2(e) / sqrt(D)
 };
 
@@ -85,7 +87,8 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Rotate the pairs of one 128 x 128 bf16 tile in place.  Row r is token n0+r.
+// Rotate the pairs of one 128 x 128 bf16 tile in place, each result rounded
+// exactly to bf16.  Row r is token n0+r; rows at or past N stay untouched.
 __device__ __forceinline__ void rotate_tile(uint8_t* tile, int n0, const Params& p, int pt) {
   for (int c = pt; c < kChunks; c += kProThreads) {
     int off, row, col0;
@@ -96,17 +99,11 @@ __device__ __forceinline__ void rotate_tile(uint8_t* tile, int n0, const Params&
     const int j0 = n * (kHeadDim / 2) + (col0 >> 1);
     const float4 cs = __ldg(reinterpret_cast<const float4*>(p.cos + j0));
     const float4 sn = __ldg(reinterpret_cast<const float4*>(p.sin + j0));
-    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    const float cc[4] = {cs.x, cs.y, cs.z, cs.w};
-    const float ss[4] = {sn.x, sn.y, sn.z, sn.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float a = bf16_lo(w[e]), b = bf16_hi(w[e]);
-      const float ra = fmaf(a, cc[e], -b * ss[e]);
-      const float rb = fmaf(a, ss[e], b * cc[e]);
-      w[e] = pack_bf16(ra, rb);
-    }
-    *reinterpret_cast<uint4*>(tile + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    x.x = rotate_pair_bf16(x.x, cs.x, sn.x);
+    x.y = rotate_pair_bf16(x.y, cs.y, sn.y);
+    x.z = rotate_pair_bf16(x.z, cs.z, sn.z);
+    x.w = rotate_pair_bf16(x.w, cs.w, sn.w);
+    *reinterpret_cast<uint4*>(tile + off) = x;
   }
 }
 
@@ -268,9 +265,13 @@ __device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, const CU
       for (int i = 0; i < 32; ++i) {
         const float p0 = ex2_approx(fmaf(f[64 * h + 2 * i], c, neg));
         const float p1 = ex2_approx(fmaf(f[64 * h + 2 * i + 1], c, neg));
-        sum0 += p0;
-        sum1 += p1;
         pk[i] = pack_f16(p0, p1);
+        // l sums the fp16-rounded P the MMA multiplies V with, so a row
+        // dominated by one key returns that key's V row exactly
+        if (i & 1)
+          sum1 = add_f16x2_to_f32(sum1, pk[i]);
+        else
+          sum0 = add_f16x2_to_f32(sum0, pk[i]);
       }
       tmem_st32(tS + 32 * h, pk);
     }
@@ -345,7 +346,7 @@ __device__ __forceinline__ void prologue_role(Smem& sm, const Params& p, const C
       const int s = j % kStages;
       const uint32_t ph = (j / kStages) & 1;
       if (!warp_wait(&sm.k_full[s], ph, wc)) break;
-      if (rope) rotate_tile(sm.k[s], j * kTile, p, pt);
+      if (rope && p.rotate_k) rotate_tile(sm.k[s], j * kTile, p, pt);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.k_ready[s]);
@@ -453,6 +454,7 @@ int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   p.n_kv = p.n_qtiles;
   p.pairs = (p.n_qtiles + 1) / 2;
   p.out_f32 = a.out_f32 ? 1 : 0;
+  p.rotate_k = (a.cos != nullptr && !a.k_rotated) ? 1 : 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kHeadDim));
   const size_t smem = sizeof(Smem) + 1024;
   static thread_local int configured_device = -1;

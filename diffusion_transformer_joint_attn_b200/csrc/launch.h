@@ -21,6 +21,15 @@ struct RopeTableArgs {
 };
 cudaError_t launch_rope_table(const RopeTableArgs& a, cudaStream_t s);
 
+struct RopeApplyArgs {
+  const void* x;
+  const float* cos;
+  const float* sin;
+  void* y;
+  int B, H, N, D;
+};
+cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t s);
+
 struct AttnFwdArgs {
   const void* q;
   const void* k;
@@ -31,6 +40,7 @@ struct AttnFwdArgs {
   float* lse;
   int B, H, N;
   bool out_f32;
+  bool k_rotated;   // k already carries the rotary embedding: rotate q only
 };
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.

@@ -249,6 +249,16 @@ __device__ __forceinline__ void regs_decrease() {
 }
 
 // ---------------------------------------------------------------- math
+// acc + lo + hi for the two fp16 halves of `packed`, each widened exactly.
+__device__ __forceinline__ float add_f16x2_to_f32(float acc, uint32_t packed) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\t"
+      "add.rn.f32.f16 %0, hi, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(packed));
+  return acc;
+}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

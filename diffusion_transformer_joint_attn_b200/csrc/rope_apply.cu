@@ -1,0 +1,42 @@
+// x_rot = R(pos) x for bf16 x [B][H][N][D]: every channel pair turned by the
+// table's (cos, sin) of its token and rounded exactly to bf16.  Memory-bound:
+// each 16-byte chunk (4 pairs) is read once and written once; the table rows
+// (N x 512 bytes) are shared by all B x H heads and stay in L2.
+#include "launch.h"
+#include "rope_exact.cuh"
+
+namespace dit {
+
+__global__ void __launch_bounds__(256) rope_apply_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
+                                                         const float* __restrict__ ts, uint4* __restrict__ y,
+                                                         long long chunks, int N) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks; c += stride) {
+    const long long row = c >> 4;                 // 16 chunks of 8 channels per token row
+    const int n = static_cast<int>(row % N);
+    const int j0 = n * 64 + static_cast<int>(c & 15) * 4;
+    const uint4 v = __ldg(x + c);
+    const float4 cs = __ldg(reinterpret_cast<const float4*>(tc + j0));
+    const float4 sn = __ldg(reinterpret_cast<const float4*>(ts + j0));
+    uint4 o;
+    o.x = rotate_pair_bf16(v.x, cs.x, sn.x);
+    o.y = rotate_pair_bf16(v.y, cs.y, sn.y);
+    o.z = rotate_pair_bf16(v.z, cs.z, sn.z);
+    o.w = rotate_pair_bf16(v.w, cs.w, sn.w);
+    y[c] = o;
+  }
+}
+
+cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t s) {
+  const long long chunks = static_cast<long long>(a.B) * a.H * a.N * (a.D / 8);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long blocks = (chunks + 255) / 256;
+  const long long cap = static_cast<long long>(sms) * 8;     // 8 resident 256-thread blocks per SM
+  if (blocks > cap) blocks = cap;
+  rope_apply_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<const uint4*>(a.x), a.cos, a.sin,
+                                                                  static_cast<uint4*>(a.y), chunks, a.N);
+  return cudaGetLastError();
+}
+
+}  // namespace dit

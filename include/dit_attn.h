@@ -54,7 +54,8 @@ typedef enum {
 
 /* Element type of q/k/v, OR-able with the flags below. */
 typedef enum { DIT_BF16 = 0, DIT_FP8_E4M3 = 1 } dit_dtype_t;
-#define DIT_OUT_F32 0x100 /* write `out` as fp32 instead of bf16 */
+#define DIT_OUT_F32 0x100   /* write `out` as fp32 instead of bf16 */
+#define DIT_K_ROTATED 0x200 /* k already carries the rotary embedding (dit_rope_apply); rotate q only */
 
 /*
  * dit_rope_table_build — cos/sin table of the three-axis rotary embedding.
@@ -79,6 +80,25 @@ int dit_rope_table_build(const int32_t* pos, int N, int D, const int32_t* axes, 
                          float* rope_sin, dit_stream_t stream);
 
 /*
+ * dit_rope_apply — x_rot = R(pos) x for bf16 x [B][H][N][D] (the rotation of
+ * dit_attn_forward, as a separate memory-bound pass).
+ *
+ *   x         device bf16 [B][H][N][D].
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2] from dit_rope_table_build.
+ *   x_rot     device bf16 [B][H][N][D], written; may equal x (in place).
+ *   B, H, N   >= 1;  D must be 128.
+ * Each rotated component is the bf16 nearest (ties to even) to the exact
+ * value x_2j*cos - x_2j+1*sin (resp. x_2j*sin + x_2j+1*cos) of the fp32 table
+ * entries, so dit_attn_forward(q, dit_rope_apply(k), ..., DIT_K_ROTATED)
+ * returns bit-for-bit what dit_attn_forward(q, k, ...) does.  Rotating K
+ * once here instead of once per query tile inside the attention kernel is the
+ * faster composition for long sequences.  All pointers 16-byte aligned.
+ */
+int dit_rope_apply(const void* x, const float* rope_cos, const float* rope_sin, void* x_rot, int B, int H, int N,
+                   int D, dit_stream_t stream);
+
+/*
  * dit_attn_forward — joint attention forward, BF16 in, BF16 (or fp32) out.
  *
  *   q, k, v   device bf16 [B][H][N][D], N = N_txt + N_img.
@@ -95,12 +115,14 @@ int dit_rope_table_build(const int32_t* pos, int N, int D, const int32_t* axes, 
  *             token attends to all N tokens (no mask); positions enter only
  *             through the tables.
  *   D         head dimension; must be 128.
- *   dtype     DIT_BF16, optionally | DIT_OUT_F32.
+ *   dtype     DIT_BF16, optionally | DIT_OUT_F32 and | DIT_K_ROTATED (the
+ *             latter requires the tables: they are then applied to q only).
  *
- * Precision: the rotation runs in fp32 and the rotated q, k are rounded to
- * bf16 tensor-core operands; q~ k~^T accumulates in fp32; the softmax runs in
- * fp32; P (in [0, 256]) and v are fp16 tensor-core operands (v must satisfy
- * |v| <= 65504), P v accumulates in fp32.
+ * Precision: each rotated component of q and k is the bf16 nearest to its
+ * exact value for the fp32 table entries; q~ k~^T accumulates in fp32; the
+ * softmax runs in fp32; P (in [0, 256]) and v are fp16 tensor-core operands
+ * (v must satisfy |v| <= 65504; the bf16 -> fp16 conversion of v is exact for
+ * |v| >= 2^-14), P v accumulates in fp32.
  * All pointers 16-byte aligned except lse (4-byte).  Graph-capturable: one
  * kernel launch, no host synchronisation, no allocation.
  */

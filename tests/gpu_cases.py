@@ -51,6 +51,11 @@ def run_gpu(w, rope=True, out_f32=False, seed=0, inputs=None):
     return out, lse
 
 
-def oracle_rows(w, q, k, v, rows, rope=True, round_rotated=None):
+def oracle_rows(w, q, k, v, rows, rope=True, operands="exact"):
+    """operands="exact": rotation and attention in fp64 on the bf16 inputs.
+    operands="bf16": rotated with the fp32 table entries and rounded to bf16,
+    the precision the kernel's tensor cores take the rotated q, k in."""
     pos = W.positions(w) if rope else None
-    return oracle_attention.joint_attention(q, k, v, pos=pos, rows=rows, round_rotated=round_rotated)
+    if operands == "exact":
+        return oracle_attention.joint_attention(q, k, v, pos=pos, rows=rows)
+    return oracle_attention.joint_attention(q, k, v, pos=pos, rows=rows, round_rotated="bf16", table_fp32=True)

@@ -6,8 +6,8 @@ Bars: max-abs <= 2e-2 and mean-abs <= 2e-3 on every checked output element,
 * Workloads with N(0,1) inputs: the bf16 output is compared with the exact
   oracle (rotation and attention in fp64 on the bf16 inputs).
 * Workloads with x16 outlier channels (logit std ~45): the fp32 output is
-  compared with the oracle whose rotated q, k are rounded to bf16, the
-  kernel's tensor-core operand precision.  With logits that large, that
+  compared with the oracle whose q, k are rotated with the fp32 table entries
+  and rounded to bf16, the kernel's tensor-core operand precision.  With logits that large, that
   operand rounding alone moves O by up to ~8 against the exact oracle, and
   rounding O itself to bf16 costs ~0.12; both are reported, not gated.
 """
@@ -67,7 +67,7 @@ def test_parity_plain_workloads(name):
     # it is gated against the operand-rounded oracle below
     check(out, lse, rows, O_ref, L_ref, name + " bf16-out vs exact", gate_lse=False)
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
-    O_op, L_op = oracle_rows(w, q, k, v, rows, round_rotated="bf16")
+    O_op, L_op = oracle_rows(w, q, k, v, rows, operands="bf16")
     check(out32, lse32, rows, O_op, L_op, name + " fp32-out vs bf16-operand oracle")
 
 
@@ -77,7 +77,7 @@ def test_parity_outlier_workloads(name):
     inputs = device_inputs(w)
     q, k, v = inputs[:3]
     rows = W.sample_rows(w)
-    O_op, L_op = oracle_rows(w, q, k, v, rows, round_rotated="bf16")
+    O_op, L_op = oracle_rows(w, q, k, v, rows, operands="bf16")
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
     check(out32, lse32, rows, O_op, L_op, name + " fp32-out vs bf16-operand oracle")
     # reported only: the format floors against the exact oracle
@@ -108,7 +108,7 @@ def test_parity_ragged_shapes(B, H, n_txt, grids):
     out, lse = run_gpu(w, inputs=inputs)
     check(out, lse, rows, O_ref, L_ref, "ragged N=%d bf16-out" % w.N, gate_lse=False)
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
-    O_op, L_op = oracle_rows(w, q, k, v, rows, round_rotated="bf16")
+    O_op, L_op = oracle_rows(w, q, k, v, rows, operands="bf16")
     check(out32, lse32, rows, O_op, L_op, "ragged N=%d fp32-out" % w.N)
 
 
@@ -120,6 +120,36 @@ def test_parity_without_rope():
     O_ref, L_ref = oracle_rows(w, q, k, v, rows, rope=False)
     out32, lse32 = run_gpu(w, rope=False, out_f32=True, inputs=inputs)
     check(out32, lse32, rows, O_ref, L_ref, "no rope fp32-out")
+
+
+def test_rope_apply_is_exactly_rounded():
+    from oracle import formats
+    w = W.WORKLOADS["t2i_2048px"]
+    q, _, _, qd, _, _ = device_inputs(w)
+    c, s = dit.rope_table(torch.from_numpy(W.positions(w)).cuda())
+    out = torch.empty_like(qd)
+    dit.dit_rope_apply(qd, c, s, out)
+    torch.cuda.synchronize()
+    rc, rs = oracle_rope.table_fp32(W.positions(w))
+    ref = formats.round_bf16(oracle_rope.rotate_with_table(q[0].double().numpy(), rc, rs))
+    got = out[0].double().cpu().numpy()
+    assert np.count_nonzero(got != ref) == 0
+    # in place gives the same
+    dit.dit_rope_apply(qd, c, s, qd)
+    assert torch.equal(qd, out)
+
+
+@pytest.mark.parametrize("name", ["tiny_256", "t2i_2048px"])
+def test_prerotated_k_matches_fused_rotation_bitwise(name):
+    w = W.WORKLOADS[name]
+    _, _, _, qd, kd, vd = device_inputs(w)
+    c, s = dit.rope_table(torch.from_numpy(W.positions(w)).cuda())
+    a, la = dit.forward(qd, kd, vd, c, s, n_txt=w.n_txt)
+    kr = torch.empty_like(kd)
+    dit.dit_rope_apply(kd, c, s, kr)
+    b, lb = dit.forward(qd, kr, vd, c, s, n_txt=w.n_txt, k_rotated=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
 
 
 def test_lse_may_be_omitted():
