@@ -1,0 +1,387 @@
+"""Benchmark of the joint text+image attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {native,reference}]
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
+
+One step is the whole BF16 hot path for one DiT attention call of the
+2048x2048-image workload (B=1, H=24, D=128, 512 text + 128x128 image tokens):
+rotary table build, the K rotation pass and the attention forward writing bf16
+O and the LSE.  Throughput is the dense attention work 4 N^2 D H B per step
+over the step time (TFLOP/s).  Each rank runs its own copy of the workload
+(weak scaling, no data-path collective); the whole-job value divides the work
+of all ranks by the slowest rank's time.
+
+`--impl reference` times the fp64 CPU oracle (the reference arm: there is no
+other implementation of this path) on a bounded sample of query rows of the
+same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+WORKLOAD = "t2i_2048px"
+METRIC = "joint-attention TFLOP/s and % of B200 dense BF16/FP8 tensor peak (1 GPU)"
+UNIT = "TFLOP/s"
+FALLBACK_PEAK_BF16 = 1590.0
+
+
+# ------------------------------------------------------------------ multi-rank
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over all ranks (x itself with one rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def whole_job_throughput(flops_per_step_per_rank: float, steps: int, world: int, max_ms: float) -> float:
+    """TFLOP/s of the whole job: work of all ranks over the slowest rank's time."""
+    return flops_per_step_per_rank * steps * world / (max_ms * 1e-3) / 1e12
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML in a thread."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks rather than fail
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        reasons = set()
+        for _, r, _ in loaded:
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    return FALLBACK_PEAK_BF16, "fallback 1.59 PFLOP/s"
+
+
+def profile_traffic(kernel_source_sha: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, or None if none exists for the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_sha") != kernel_source_sha or d.get("workload") != WORKLOAD:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+    csrc = os.path.join(ROOT, "diffusion_transformer_joint_attn_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def oracle_sample(w, rows_per_head: int):
+    """Rows (b, h, n) of the CPU-baseline sample: the first rows_per_head query
+    rows of every head."""
+    rows = [(b, h, n) for b in range(w.B) for h in range(w.H) for n in range(rows_per_head)]
+    return np.asarray(rows, dtype=np.int64)
+
+
+def time_oracle(w, q, k, v, rows):
+    from oracle import attention as oracle_attention
+    from threadpoolctl import threadpool_info
+    t0 = time.perf_counter()
+    oracle_attention.joint_attention(q, k, v, pos=W.positions(w), rows=rows)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    flops = 4.0 * w.N * w.D * len(rows)
+    return flops / dt / 1e12, dt, threads
+
+
+# ------------------------------------------------------------------ native arm
+def run_native(args):
+    import torch
+    import diffusion_transformer_joint_attn_b200 as dit
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = W.WORKLOADS[args.workload]
+    dit.load_library()
+
+    q_h, k_h, v_h = W.make_qkv(w, seed=rank)
+    pos_h = torch.from_numpy(W.positions(w))
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    pos = pos_h.to(dev)
+    cos = torch.empty((w.N, 64), dtype=torch.float32, device=dev)
+    sin = torch.empty_like(cos)
+    k_rot = torch.empty_like(k)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = dit.load_library()
+    s_ptr = stream.cuda_stream
+    axes = (ctypes.c_int32 * 3)(*W.ROPE_AXES)
+    flags = dit.DIT_BF16 | dit.DIT_K_ROTATED
+
+    def step(ev=None):
+        # the whole BF16 hot path: rotary table, K rotation, attention forward
+        assert lib.dit_rope_table_build(pos.data_ptr(), w.N, w.D, axes, W.ROPE_THETA, cos.data_ptr(),
+                                        sin.data_ptr(), s_ptr) == 0
+        assert lib.dit_rope_apply(k.data_ptr(), cos.data_ptr(), sin.data_ptr(), k_rot.data_ptr(), w.B, w.H, w.N,
+                                  w.D, s_ptr) == 0
+        if ev is not None:
+            ev[0].record(stream)
+        assert lib.dit_attn_forward(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(), cos.data_ptr(), sin.data_ptr(),
+                                    out.data_ptr(), lse.data_ptr(), w.B, w.H, w.n_txt, w.n_img, w.D, flags,
+                                    s_ptr) == 0
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = dit.dit_attn_get_status(stream)
+    if status != 0:
+        raise RuntimeError("device status %d after warm-up" % status)
+
+    kern_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(kern_ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    kern_ms = sum(a.elapsed_time(b) for a, b in kern_ev) / args.steps
+    if dit.dit_attn_get_status(stream) != 0:
+        raise RuntimeError("device status error in the timed region")
+    max_ms = max_over_ranks(ms, world, dev)
+    value = whole_job_throughput(w.flops, args.steps, world, max_ms)
+
+    # end to end through the public API: pinned host inputs in, O and LSE out
+    q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    pos_p = pos_h.pin_memory()
+    out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (q_p, k_p, v_p, pos_p))
+    d2h = out_p.numel() * out_p.element_size() + lse_p.numel() * lse_p.element_size()
+
+    def e2e_step():
+        q.copy_(q_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        pos.copy_(pos_p, non_blocking=True)
+        step()
+        out_p.copy_(out, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_throughput(w.flops, e2e_steps, world, e2e_ms)
+
+    peak, peak_src = measured_peaks()
+    achieved = w.flops / (kern_ms * 1e-3) / 1e12
+    traffic = profile_traffic(kernel_source_sha()) if w.name == WORKLOAD else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = oracle_sample(w, args.oracle_rows_per_head)
+        val, dt, threads = time_oracle(w, q_h, k_h, v_h, rows)
+        cpu = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "fp64 numpy oracle on the first %d query rows of each of the %d heads (%d rows of %d, "
+                         "%.1f s)" % (args.oracle_rows_per_head, w.H * w.B, len(rows), w.B * w.H * w.N, dt)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "n_txt": w.n_txt, "n_img": w.n_img,
+                       "N": w.N, "inputs": "seeded N(0,1) bf16, channels 3/40/77/110 x16",
+                       "step": "rope table + K rotation + attention forward (bf16 O, fp32 LSE)",
+                       "l2": "inputs larger than L2 (q, k, v %.0f MB > 126 MB), no flush" % (6 * w.B * w.H * w.N * w.D / 1e6),
+                       "parallelism": "replica per GPU" if world > 1 else "single GPU",
+                       "pct_of_bf16_peak": 100.0 * value / peak},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "attn_fwd_bf16_kernel", "peak_source": peak_src,
+                         "kernel_ms": kern_ms},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / e2e_steps},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The fp64 oracle on the host cores: step i evaluates the first
+    --reference-rows query rows of head i mod H of the same workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = W.WORKLOADS[WORKLOAD]
+    q, k, v = W.make_qkv(w, seed=0)
+    R = args.reference_rows
+
+    def rows_of(i):
+        h = i % w.H
+        return np.asarray([(0, h, n) for n in range(R)], dtype=np.int64)
+
+    for i in range(args.warmup):
+        time_oracle(w, q, k, v, rows_of(i))
+    total = 0.0
+    threads = 1
+    for i in range(args.steps):
+        _, dt, threads = time_oracle(w, q, k, v, rows_of(i))
+        total += dt
+    flops = 4.0 * w.N * w.D * R
+    value = flops * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "D": w.D, "n_txt": w.n_txt, "n_img": w.n_img, "N": w.N},
+        "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": threads,
+                         "sample": "fp64 numpy oracle: per step the first %d query rows of one head (heads in turn)"
+                                   % R},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=W.ORDER, default=WORKLOAD,
+                    help="the bench line is the default workload; others serve profiling")
+    ap.add_argument("--oracle-rows-per-head", type=int, default=2048)
+    ap.add_argument("--reference-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()
