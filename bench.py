@@ -206,23 +206,24 @@ def run_native(args):
     cos = torch.empty((w.N, 64), dtype=torch.float32, device=dev)
     sin = torch.empty_like(cos)
     k_rot = torch.empty_like(k)
+    v_f16 = torch.empty(v.shape, dtype=torch.float16, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     lib = dit.load_library()
     s_ptr = stream.cuda_stream
     axes = (ctypes.c_int32 * 3)(*W.ROPE_AXES)
-    flags = dit.DIT_BF16 | dit.DIT_K_ROTATED
+    flags = dit.DIT_BF16 | dit.DIT_K_ROTATED | dit.DIT_V_F16
 
     def step(ev=None):
-        # the whole BF16 hot path: rotary table, K rotation, attention forward
+        # the whole BF16 hot path: rotary table, K / V operand pass, attention forward
         assert lib.dit_rope_table_build(pos.data_ptr(), w.N, w.D, axes, W.ROPE_THETA, cos.data_ptr(),
                                         sin.data_ptr(), s_ptr) == 0
-        assert lib.dit_rope_apply(k.data_ptr(), cos.data_ptr(), sin.data_ptr(), k_rot.data_ptr(), w.B, w.H, w.N,
-                                  w.D, s_ptr) == 0
+        assert lib.dit_attn_prepare_kv(k.data_ptr(), v.data_ptr(), cos.data_ptr(), sin.data_ptr(), k_rot.data_ptr(),
+                                       v_f16.data_ptr(), w.B, w.H, w.N, w.D, s_ptr) == 0
         if ev is not None:
             ev[0].record(stream)
-        assert lib.dit_attn_forward(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(), cos.data_ptr(), sin.data_ptr(),
+        assert lib.dit_attn_forward(q.data_ptr(), k_rot.data_ptr(), v_f16.data_ptr(), cos.data_ptr(), sin.data_ptr(),
                                     out.data_ptr(), lse.data_ptr(), w.B, w.H, w.n_txt, w.n_img, w.D, flags,
                                     s_ptr) == 0
         if ev is not None:
@@ -306,7 +307,7 @@ def run_native(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "n_txt": w.n_txt, "n_img": w.n_img,
                        "N": w.N, "inputs": "seeded N(0,1) bf16, channels 3/40/77/110 x16",
-                       "step": "rope table + K rotation + attention forward (bf16 O, fp32 LSE)",
+                       "step": "rope table + K/V operand pass + attention forward (bf16 O, fp32 LSE)",
                        "l2": "inputs larger than L2 (q, k, v %.0f MB > 126 MB), no flush" % (6 * w.B * w.H * w.N * w.D / 1e6),
                        "parallelism": "replica per GPU" if world > 1 else "single GPU",
                        "pct_of_bf16_peak": 100.0 * value / peak},

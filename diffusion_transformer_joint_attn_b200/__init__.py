@@ -23,6 +23,7 @@ DIT_BF16 = 0
 DIT_FP8_E4M3 = 1
 DIT_OUT_F32 = 0x100
 DIT_K_ROTATED = 0x200
+DIT_V_F16 = 0x400
 
 
 class DitError(RuntimeError):
@@ -80,6 +81,21 @@ def dit_rope_apply(x, rope_cos, rope_sin, x_rot, stream=None) -> None:
                                          _stream(stream)), "dit_rope_apply")
 
 
+def dit_attn_prepare_kv(k, v, rope_cos, rope_sin, k_rot, v_f16, stream=None) -> None:
+    """k_rot <- rotated bf16 k, v_f16 <- fp16 copy of v (both [B, H, N, D])."""
+    import torch
+    _require(k.dim() == 4 and k.shape == v.shape == k_rot.shape == v_f16.shape, "k, v, k_rot, v_f16 shapes differ")
+    B, H, N, D = k.shape
+    for t in (k, v, k_rot):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "k, v, k_rot must be contiguous CUDA bf16")
+    _require(v_f16.is_cuda and v_f16.dtype == torch.float16 and v_f16.is_contiguous(), "v_f16 must be CUDA fp16")
+    for t in (rope_cos, rope_sin):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (N, D // 2),
+                 "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _check(load_library().dit_attn_prepare_kv(_ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(k_rot),
+                                              _ptr(v_f16), B, H, N, D, _stream(stream)), "dit_attn_prepare_kv")
+
+
 def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: int, dtype: int = DIT_BF16,
                      stream=None) -> None:
     """out (and lse, if not None) <- joint attention of bf16 q, k, v [B, H, N, D] on the GPU."""
@@ -87,8 +103,10 @@ def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: i
     _require(q.dim() == 4 and q.shape == k.shape == v.shape, "q, k, v must share one [B, H, N, D] shape")
     B, H, N, D = q.shape
     _require(N == n_txt + n_img, "N must equal n_txt + n_img")
-    for t in (q, k, v):
-        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "q, k, v must be contiguous CUDA bf16")
+    for t in (q, k):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "q, k must be contiguous CUDA bf16")
+    v_dtype = torch.float16 if dtype & DIT_V_F16 else torch.bfloat16
+    _require(v.is_cuda and v.dtype == v_dtype and v.is_contiguous(), "v must be contiguous CUDA bf16 (fp16 with DIT_V_F16)")
     out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
     _require(out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q.shape,
              "out must be a contiguous CUDA tensor of q's shape and the requested dtype")
@@ -127,12 +145,12 @@ def rope_table(pos, axes=(16, 56, 56), theta: float = 10000.0, stream=None):
 
 
 def forward(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool = False, with_lse: bool = True,
-            k_rotated: bool = False, stream=None):
+            k_rotated: bool = False, v_f16: bool = False, stream=None):
     """Allocate out (and lse) and run dit_attn_forward; returns (out, lse)."""
     import torch
     B, H, N, D = q.shape
     out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
-    flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0)
+    flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0) | (DIT_V_F16 if v_f16 else 0)
     dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt, DIT_BF16 | flags, stream)
     return out, lse

@@ -16,6 +16,7 @@ _I = ctypes.c_int
 SIGNATURES = {
     "dit_rope_table_build": (_I, [_VP, _I, _I, ctypes.POINTER(ctypes.c_int32), ctypes.c_double, _VP, _VP, _VP]),
     "dit_rope_apply": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
+    "dit_attn_prepare_kv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_get_status": (_I, [ctypes.POINTER(ctypes.c_int), _VP]),
     "dit_attn_status_string": (ctypes.c_char_p, [_I]),

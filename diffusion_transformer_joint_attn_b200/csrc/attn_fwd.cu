@@ -1,46 +1,67 @@
 // Joint text+image attention forward for sm_100a (BF16 in, BF16/fp32 out).
 //
-// One CTA owns two 128-row query tiles of one (b, h) and streams every
-// 128-key tile of K and V past them (flash-style online softmax), so the
-// logits never leave the SM.  Roles, by warp:
+// A cluster of two CTAs (a CTA pair on the two SMs of a TPC) owns four
+// 128-row query tiles of one (b, h): two per CTA, processed as two 256-row
+// "slots" (rows 0-127 of a slot in the even CTA, 128-255 in the odd one).
+// Every 128-key tile of K and V streams past them (flash-style online
+// softmax), so the logits never leave the SMs.  The even CTA issues pair MMAs
+// (tcgen05 cta_group::2, M = 256) that read each CTA's own Q rows and P rows
+// and half of the B operand from each CTA: keys 0-63 / 64-127 of a K tile,
+// channels 0-63 / 64-127 of a V tile.  Each SM therefore loads and reads
+// only half of every K and V tile, which keeps the shared-memory port below
+// the rate the two products need.
 //
-//   warp 0        TMA producer: Q tiles once, then K_j / V_j into 2-slot rings
-//   warp 1        MMA issuer:   S_t = Q_t K_j^T (bf16 operands, smem x smem)
-//                               O_t += P_t V_j (fp16 operands, P from TMEM)
-//   warps 2-3,    operand prologue: rotary embedding of Q (once) and of every
-//   12-15         K_j in shared memory (fp32 math, rounded to bf16), and the
-//                 exact bf16 -> fp16 conversion of every V_j
-//   warps 4-7     softmax of query tile 0 (one thread per query row)
-//   warps 8-11    softmax of query tile 1
+// Roles, by warp (in both CTAs unless stated):
+//   warp 0        TMA producer: own Q tiles once, own K_j / V_j halves into
+//                 4-slot rings
+//   warp 1        MMA issuer (even CTA only): S_t = Q_t K_j^T (bf16),
+//                 O_t += P_t V_j (fp16, P from tensor memory)
+//   warps 2-15    rotary embedding of the CTA's two Q tiles, once
+//   warps 2-3,    in-loop operand work when K / V were not prepared by
+//   12-15         dit_attn_prepare_kv: rotation of the K_j half and the exact
+//                 bf16 -> fp16 conversion of the V_j half, in shared memory
+//   warps 4-7     softmax of slot 0 (one thread per query row)
+//   warps 8-11    softmax of slot 1
 //
-// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1, each 128 lanes x 128
-// fp32 columns; P_t (fp16) overwrites the first 64 columns of S_t.  While the
-// softmax warps of one tile work, the tensor core runs the other tile's MMAs.
-#include <cstdio>
-
+// Tensor memory per CTA (512 columns): S_0 | S_1 | O_0 | O_1, 128 lanes x 128
+// fp32 columns each; P_t (fp16) overwrites the first 64 columns of S_t.
+// While the softmax warps of one slot work, the tensor cores run the other
+// slot's MMAs.
 #include "launch.h"
 #include "ptx.cuh"
 #include "rope_exact.cuh"
+#include "softmax_exp2.cuh"
 
 namespace dit {
 namespace {
 
-constexpr int kTile = 128;                  // query rows per tile = keys per tile
+constexpr int kTile = 128;                         // query rows per tile = keys per K/V tile
 constexpr int kHeadDim = 128;
-constexpr int kStages = 2;                  // K and V ring depth
-constexpr int kTileBytes = kTile * kHeadDim * 2;   // 32 KB
-constexpr int kBoxBytes = kTile * 64 * 2;          // 16 KB: 128 rows x 64 channels
+constexpr int kStages = 4;                         // K and V ring depth
+constexpr int kQTileBytes = kTile * kHeadDim * 2;  // 32 KB: 128 rows x 128 channels
+constexpr int kQBoxBytes = kTile * 64 * 2;         // 16 KB: 128 rows x 64 channels
+constexpr int kKHalfBytes = 64 * kHeadDim * 2;     // 16 KB: 64 keys x 128 channels
+constexpr int kKBoxBytes = 64 * 64 * 2;            // 8 KB: 64 keys x 64 channels
+constexpr int kVHalfBytes = kTile * 64 * 2;        // 16 KB: 128 keys x 64 channels
 constexpr int kThreads = 512;
-constexpr int kProWarps = 6;
+constexpr int kProWarps = 6;                       // in-loop operand warps per CTA
 constexpr int kProThreads = kProWarps * 32;
-constexpr int kChunks = kTileBytes / 16;           // 16-byte chunks per tile
+constexpr int kQRotThreads = 14 * 32;              // warps 2-15 rotate Q
+constexpr int kBarQRot = 1;                        // named barrier of the Q rotation
+constexpr int kPolyEvery = 4;                      // every kPolyEvery-th exponent pair on the FMA pipe (0: none)
+// Register split of the 4 x 128 x 128 launch registers between warpgroups:
+// producer / MMA warpgroup, the two softmax warpgroups, the operand warpgroup.
+constexpr uint32_t kIssueRegs = 80;
+constexpr uint32_t kSoftmaxRegs = 184;
+constexpr uint32_t kOperandRegs = 64;
+static_assert(kIssueRegs + 2 * kSoftmaxRegs + kOperandRegs == 4 * 128, "register split must use the launch budget");
 
 struct __align__(1024) Smem {
-  uint8_t q[2][kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t q[2][kQTileBytes];
+  uint8_t k[kStages][kKHalfBytes];
+  uint8_t v[kStages][kVHalfBytes];
   uint64_t q_full;
-  uint64_t q_ready;
+  uint64_t q_ready;                                   // even CTA: one arrive per CTA
   uint64_t k_full[kStages], k_ready[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_ready[kStages], v_empty[kStages];
   uint64_t s_full[2], p_ready[2], o_final[2];
@@ -56,61 +77,93 @@ struct Params {
   float* lse;
   int* status;
   int N;
-  int n_qtiles;
   int n_kv;
-  int pairs;          // query-tile pairs per (b, h)
+  int clusters;       // CTA pairs per (b, h): 512 query rows each
   int out_f32;
-  int rotate_k;       // rotate K tiles in the kernel (0: K arrives rotated or no rotary embedding)
+  int rotate_k;       // rotate K halves in the loop
+  int convert_v;      // convert V halves bf16 -> fp16 in the loop
   float scale_log2;   // log2(e) / sqrt(D)
 };
 
-// Byte offset, inside a tile, of 16-byte chunk `c` (0..2047) of the physical
-// layout the 128-byte-swizzled TMA boxes produce, and the tile coordinates
-// (row, first channel) whose 8 values it holds.
-__device__ __forceinline__ void chunk_coords(int c, int& byte_off, int& row, int& col0) {
-  const int box = c >> 10;          // channels 0-63 | 64-127
+struct Pair {
+  uint32_t rank;      // 0: even (MMA-issuing) CTA, 1: odd CTA
+  uint32_t peer;
+  int bh;
+  int row0[2];        // first query row of this CTA's tile in slot 0 / 1
+};
+
+// shared::cluster address of `p` in CTA `rank` of the pair.
+__device__ __forceinline__ uint32_t cl(const void* p, uint32_t rank) { return mapa_shared(smem_u32(p), rank); }
+
+// Q tile chunk c (0..2047): byte offset in the 128B-swizzled layout of two
+// 128-row x 64-channel boxes, its row and first channel.
+__device__ __forceinline__ void q_chunk(int c, int& byte_off, int& row, int& col0) {
+  const int box = c >> 10;
   row = (c >> 3) & 127;
   const int phys = c & 7;
-  const int logical = phys ^ (row & 7);
-  byte_off = box * kBoxBytes + row * 128 + phys * 16;
-  col0 = box * 64 + logical * 8;
+  byte_off = box * kQBoxBytes + row * 128 + phys * 16;
+  col0 = box * 64 + ((phys ^ (row & 7)) << 3);
+}
+// K half-tile chunk c (0..1023): two 64-row x 64-channel boxes.
+__device__ __forceinline__ void k_chunk(int c, int& byte_off, int& row, int& col0) {
+  const int box = c >> 9;
+  row = (c >> 3) & 63;
+  const int phys = c & 7;
+  byte_off = box * kKBoxBytes + row * 128 + phys * 16;
+  col0 = box * 64 + ((phys ^ (row & 7)) << 3);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Rotate the pairs of one 128 x 128 bf16 tile in place, each result rounded
-// exactly to bf16.  Row r is token n0+r; rows at or past N stay untouched.
-__device__ __forceinline__ void rotate_tile(uint8_t* tile, int n0, const Params& p, int pt) {
-  for (int c = pt; c < kChunks; c += kProThreads) {
-    int off, row, col0;
-    chunk_coords(c, off, row, col0);
-    const int n = n0 + row;
-    if (n >= p.N) continue;
-    uint4 x = *reinterpret_cast<const uint4*>(tile + off);
-    const int j0 = n * (kHeadDim / 2) + (col0 >> 1);
-    const float4 cs = __ldg(reinterpret_cast<const float4*>(p.cos + j0));
-    const float4 sn = __ldg(reinterpret_cast<const float4*>(p.sin + j0));
-    x.x = rotate_pair_bf16(x.x, cs.x, sn.x);
-    x.y = rotate_pair_bf16(x.y, cs.y, sn.y);
-    x.z = rotate_pair_bf16(x.z, cs.z, sn.z);
-    x.w = rotate_pair_bf16(x.w, cs.w, sn.w);
-    *reinterpret_cast<uint4*>(tile + off) = x;
+// Rotate chunks first, first+kStep, ... (< kChunks) of a tile whose row r is
+// token n0 + r, in place, each component rounded exactly to bf16.  The loads
+// of kBatch chunks are issued before any of them is used.
+template <int kChunks, int kStep, int kBatch, bool kHalfK>
+__device__ __forceinline__ void rotate_chunks(uint8_t* tile, int n0, const Params& p, int first) {
+  for (int c0 = first; c0 < kChunks; c0 += kBatch * kStep) {
+    uint4 x[kBatch];
+    float4 cs[kBatch], sn[kBatch];
+    int off[kBatch];
+    bool live[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + u * kStep;
+      int row, col0;
+      if (kHalfK)
+        k_chunk(c < kChunks ? c : 0, off[u], row, col0);
+      else
+        q_chunk(c < kChunks ? c : 0, off[u], row, col0);
+      const int n = n0 + row;
+      live[u] = c < kChunks && n < p.N;
+      if (live[u]) {
+        const int j0 = n * (kHeadDim / 2) + (col0 >> 1);
+        x[u] = *reinterpret_cast<const uint4*>(tile + off[u]);
+        cs[u] = __ldg(reinterpret_cast<const float4*>(p.cos + j0));
+        sn[u] = __ldg(reinterpret_cast<const float4*>(p.sin + j0));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (!live[u]) continue;
+      uint4 y;
+      y.x = rotate_pair_bf16(x[u].x, cs[u].x, sn[u].x);
+      y.y = rotate_pair_bf16(x[u].y, cs[u].y, sn[u].y);
+      y.z = rotate_pair_bf16(x[u].z, cs[u].z, sn[u].z);
+      y.w = rotate_pair_bf16(x[u].w, cs[u].w, sn[u].w);
+      *reinterpret_cast<uint4*>(tile + off[u]) = y;
+    }
   }
 }
 
-// bf16 -> fp16 in place (exact for |x| in [2^-14, 65504]; below that the
-// fp16 subnormal spacing 2^-24 bounds the error).
-__device__ __forceinline__ void convert_tile_f16(uint8_t* tile, int pt) {
-  for (int c = pt; c < kChunks; c += kProThreads) {
+// bf16 -> fp16 in place for a V half tile (exact for |x| in [2^-14, 65504];
+// below that the fp16 subnormal spacing 2^-24 bounds the error).
+__device__ __forceinline__ void convert_half_f16(uint8_t* tile, int pt) {
+  for (int c = pt; c < kVHalfBytes / 16; c += kProThreads) {
     uint4* ptr = reinterpret_cast<uint4*>(tile + c * 16);
     uint4 x = *ptr;
     x.x = pack_f16(bf16_lo(x.x), bf16_hi(x.x));
@@ -121,105 +174,187 @@ __device__ __forceinline__ void convert_tile_f16(uint8_t* tile, int pt) {
   }
 }
 
-// TMA producer (warp 0).
-__device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v, uint32_t tmem, int bh, int q0, int warp, int lane, const WaitCtx& wc) {
-  if (lane == 0) {
-    tma_prefetch_desc(tm_q);
-    tma_prefetch_desc(tm_k);
-    tma_prefetch_desc(tm_v);
-    mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
-    for (int t = 0; t < 2; ++t)
-      for (int b = 0; b < 2; ++b) tma_load_3d(sm.q[t] + b * kBoxBytes, tm_q, &sm.q_full, b * 64, q0 + t * kTile, bh);
-    int issued = 0;
-    for (int j = 0; j < p.n_kv; ++j) {
-      const int s = j % kStages;
-      const uint32_t ph = (j / kStages) & 1;
-      if (!mbar_wait(&sm.k_empty[s], ph ^ 1, wc)) break;
-      mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
-      for (int b = 0; b < 2; ++b) tma_load_3d(sm.k[s] + b * kBoxBytes, tm_k, &sm.k_full[s], b * 64, j * kTile, bh);
-      if (!mbar_wait(&sm.v_empty[s], ph ^ 1, wc)) {
-        issued = 2 * j + 1;
-        break;
-      }
-      mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
-      for (int b = 0; b < 2; ++b) tma_load_3d(sm.v[s] + b * kBoxBytes, tm_v, &sm.v_full[s], b * 64, j * kTile, bh);
-      issued = 2 * j + 2;
+// ---------------------------------------------------------------- producer
+// kPrepared: K / V halves land MMA-ready; their bytes are counted on the even
+// CTA's barriers (one expect_tx there covers both halves).  Otherwise each
+// CTA counts its own halves locally for its operand warps.
+template <bool kPrepared>
+__device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v, const Pair& pr,
+                                              const WaitCtx& wc) {
+  tma_prefetch_desc(tm_q);
+  tma_prefetch_desc(tm_k);
+  tma_prefetch_desc(tm_v);
+  mbar_arrive_expect_tx(&sm.q_full, 2 * kQTileBytes);
+  for (int t = 0; t < 2; ++t)
+    for (int b = 0; b < 2; ++b)
+      tma_load_3d(sm.q[t] + b * kQBoxBytes, tm_q, &sm.q_full, b * 64, pr.row0[t], pr.bh);
+  const bool leader = pr.rank == 0;
+  int issued = 0;
+  for (int j = 0; j < p.n_kv; ++j) {
+    const int s = j % kStages;
+    const uint32_t ph = (j / kStages) & 1;
+    const int key0 = j * kTile;
+    if (!mbar_wait(&sm.k_empty[s], ph ^ 1, wc)) break;
+    if (kPrepared) {
+      if (leader) mbar_arrive_expect_tx(&sm.k_full[s], 2 * kKHalfBytes);
+      const uint32_t bar = cl(&sm.k_full[s], 0);
+      for (int b = 0; b < 2; ++b)
+        tma_load_3d_pair(sm.k[s] + b * kKBoxBytes, tm_k, bar, b * 64, key0 + 64 * static_cast<int>(pr.rank), pr.bh);
+    } else {
+      mbar_arrive_expect_tx(&sm.k_full[s], kKHalfBytes);
+      for (int b = 0; b < 2; ++b)
+        tma_load_3d(sm.k[s] + b * kKBoxBytes, tm_k, &sm.k_full[s], b * 64, key0 + 64 * static_cast<int>(pr.rank),
+                    pr.bh);
     }
-    if (*wc.abort) {
-      // let every copy already issued land before the CTA exits
-      mbar_wait_drain(&sm.q_full, 0, wc);
+    if (!mbar_wait(&sm.v_empty[s], ph ^ 1, wc)) {
+      issued = 2 * j + 1;
+      break;
+    }
+    if (kPrepared) {
+      if (leader) mbar_arrive_expect_tx(&sm.v_full[s], 2 * kVHalfBytes);
+      tma_load_3d_pair(sm.v[s], tm_v, cl(&sm.v_full[s], 0), 64 * static_cast<int>(pr.rank), key0, pr.bh);
+    } else {
+      mbar_arrive_expect_tx(&sm.v_full[s], kVHalfBytes);
+      tma_load_3d(sm.v[s], tm_v, &sm.v_full[s], 64 * static_cast<int>(pr.rank), key0, pr.bh);
+    }
+    issued = 2 * j + 2;
+  }
+  if (*wc.abort) {
+    // Let the copies already issued land before the pair exits.  Copies whose
+    // bytes the even CTA counts are drained there; the odd CTA waits out a
+    // few microseconds instead.
+    mbar_wait_drain(&sm.q_full, 0, wc);
+    if (!kPrepared || leader) {
       for (int i = (issued > 2 * kStages ? issued - 2 * kStages : 0); i < issued; ++i) {
         const int j = i / 2, s = j % kStages;
         const uint32_t ph = (j / kStages) & 1;
         mbar_wait_drain((i & 1) ? &sm.v_full[s] : &sm.k_full[s], ph, wc);
       }
-    }
-  }
-}
-
-// MMA issuer (warp 1).
-__device__ __forceinline__ void mma_role(Smem& sm, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v, uint32_t tmem, int bh, int q0, int warp, int lane, const WaitCtx& wc) {
-  if (lane == 0) {
-    constexpr uint32_t idesc_qk = instr_desc(1, 1, 128, 128, 0, 0);   // bf16 x bf16, both K-major
-    constexpr uint32_t idesc_pv = instr_desc(0, 0, 128, 128, 0, 1);   // f16 x f16, V MN-major
-    const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
-    bool ok = mbar_wait(&sm.q_ready, 0, wc);
-    tc_fence_after();
-    int j = 0;
-    for (; ok && j <= p.n_kv; ++j) {
-      const int s = j % kStages;
-      const int sp = (j + kStages - 1) % kStages;
-      for (int t = 0; t < 2 && ok; ++t) {
-        const uint32_t tS = tmem + t * 128;
-        const uint32_t tO = tmem + 256 + t * 128;
-        if (j > 0) {
-          // O_t += P_t V_{j-1}
-          if (!(ok = mbar_wait(&sm.p_ready[t], (j - 1) & 1, wc))) break;
-          if (t == 0 && !(ok = mbar_wait(&sm.v_ready[sp], ((j - 1) / kStages) & 1, wc))) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sm.v[sp]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024);
-            mma_ts(tO, tS + kk * 8, bdesc, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
-          }
-          if (j == p.n_kv) tc_commit(&sm.o_final[t]);
-        }
-        if (j < p.n_kv) {
-          // S_t = Q_t K_j^T
-          if (t == 0) {
-            if (!(ok = mbar_wait(&sm.k_ready[s], (j / kStages) & 1, wc))) break;
-            tc_fence_after();
-          }
-          const uint32_t k_addr = smem_u32(sm.k[s]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            const uint64_t adesc = smem_desc_sw128(q_addr[t] + off, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(k_addr + off, 16, 1024);
-            mma_ss(tS, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&sm.s_full[t]);
-        }
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 20000) {
       }
-      if (!ok) break;
-      if (j < p.n_kv) tc_commit(&sm.k_empty[s]);
-      if (j > 0) tc_commit(&sm.v_empty[sp]);
     }
-    // every MMA issued above has completed once this arrives
-    tc_commit(&sm.mma_drain);
-    mbar_wait_drain(&sm.mma_drain, 0, wc);
   }
 }
 
-// Online softmax and epilogue of one query tile (warps 4-11).
-__device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v, uint32_t tmem, int bh, int q0, int warp, int lane, const WaitCtx& wc) {
+// ---------------------------------------------------------------- MMA issuer
+// Even CTA only.  Completion of pair MMAs is signalled to the barrier of the
+// same name in both CTAs.
+__device__ __forceinline__ void commit_both(uint64_t* bar) {
+  tc_commit_pair(cl(bar, 0));
+  tc_commit_pair(cl(bar, 1));
+}
+
+template <bool kPrepared>
+__device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tmem, const WaitCtx& wc) {
+  constexpr uint32_t idesc_qk = instr_desc(1, 1, 256, 128, 0, 0);   // bf16 x bf16, both K-major
+  constexpr uint32_t idesc_pv = instr_desc(0, 0, 256, 128, 0, 1);   // f16 x f16, V MN-major
+  // Descriptors, built once: ring slots are contiguous, so slot s and the k-th
+  // 16-wide slice of a tile only move the start address (field in 16-byte
+  // units) by constants; no runtime-indexed arrays (they would live in local
+  // memory and stall the issuing thread).
+  const uint64_t q_desc0 = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
+  const uint64_t k_desc0 = smem_desc_sw128(smem_u32(sm.k[0]), 16, 1024);
+  const uint64_t v_desc0 = smem_desc_sw128(smem_u32(sm.v[0]), kVHalfBytes, 1024);
+  uint64_t* k_bar = kPrepared ? sm.k_full : sm.k_ready;
+  uint64_t* v_bar = kPrepared ? sm.v_full : sm.v_ready;
+  bool ok = mbar_wait(&sm.q_ready, 0, wc);
+  tc_fence_after();
+  for (int j = 0; ok && j <= p.n_kv; ++j) {
+    const int s = j % kStages;
+    const int sp = (j + kStages - 1) % kStages;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t tS = tmem + t * 128;
+      const uint32_t tO = tmem + 256 + t * 128;
+      if (j > 0) {
+        // O_t += P_t V_{j-1}
+        if (!(ok = mbar_wait(&sm.p_ready[t], (j - 1) & 1, wc))) break;
+        if (t == 0 && !(ok = mbar_wait(&v_bar[sp], ((j - 1) / kStages) & 1, wc))) break;
+        tc_fence_after();
+        const uint64_t vd = v_desc0 + static_cast<uint32_t>(sp) * (kVHalfBytes >> 4);
+        mma_ts_pair(tO, tS, vd, idesc_pv, j > 1 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk) mma_ts_pair(tO, tS + kk * 8, vd + kk * (2048 >> 4), idesc_pv, 1u);
+        if (j == p.n_kv) commit_both(&sm.o_final[t]);
+      }
+      if (j < p.n_kv) {
+        // S_t = Q_t K_j^T
+        if (t == 0) {
+          if (!(ok = mbar_wait(&k_bar[s], (j / kStages) & 1, wc))) break;
+          tc_fence_after();
+        }
+        const uint64_t qd = q_desc0 + t * (kQTileBytes >> 4);
+        const uint64_t kd = k_desc0 + static_cast<uint32_t>(s) * (kKHalfBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = ((kk >> 2) * kQBoxBytes + (kk & 3) * 32) >> 4;
+          const uint32_t boff = ((kk >> 2) * kKBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss_pair(tS, qd + aoff, kd + boff, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        commit_both(&sm.s_full[t]);
+      }
+    }
+    if (!ok) break;
+    if (j < p.n_kv) commit_both(&sm.k_empty[s]);
+    if (j > 0) commit_both(&sm.v_empty[sp]);
+  }
+  // every MMA issued above has completed once this arrives
+  tc_commit_pair(cl(&sm.mma_drain, 0));
+  mbar_wait_drain(&sm.mma_drain, 0, wc);
+}
+
+// ---------------------------------------------------------------- softmax
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Max of 64 consecutive values (4 independent chains of 3-input max).
+__device__ __forceinline__ float max64(const float* f) {
+  float m[4] = {f[0], f[1], f[2], f[3]};
+#pragma unroll
+  for (int i = 4; i < 64; i += 8) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m[u] = fmax3(m[u], f[i + 2 * u], f[i + 2 * u + 1]);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// P for 64 consecutive logits of the row: 2^(s c - m c) rounded to fp16, packed
+// in pairs into pk[32]; adds the rounded values to sum[4].
+__device__ __forceinline__ void exp_half(const float* f, float c, float neg, uint32_t* pk, float* sum) {
+  const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 x = __ffma2_rn(make_float2(f[2 * i], f[2 * i + 1]), c2, n2);
+    float e0, e1;
+    if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
+      exp2_pair_poly(x.x, x.y, e0, e1);
+    } else {
+      e0 = ex2_approx(x.x);
+      e1 = ex2_approx(x.y);
+    }
+    pk[i] = pack_f16(e0, e1);
+    // l sums the fp16-rounded P the MMA multiplies V with, so a row
+    // dominated by one key returns that key's V row exactly
+    sum[i & 3] = add_f16x2_to_f32(sum[i & 3], pk[i]);
+  }
+}
+
+// Online softmax and epilogue of this CTA's tile of one slot (warps 4-11).
+__device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, uint32_t tmem, const Pair& pr, int warp,
+                                             int lane, const WaitCtx& wc) {
   const int t = (warp - 4) >> 2;
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tS = tmem + lane_base + t * 128;
   const uint32_t tO = tmem + lane_base + 256 + t * 128;
+  const uint32_t p_ready_even = cl(&sm.p_ready[t], 0);
   const float c = p.scale_log2;
   const float rescale_gap = 8.0f / c;     // lazy rescale once the max grew by 2^8
   const int last_valid = p.N - (p.n_kv - 1) * kTile;
@@ -239,9 +374,7 @@ __device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, const CU
       for (int i = 0; i < 128; ++i)
         if (i >= last_valid) f[i] = -INFINITY;
     }
-    float mx = f[0];
-#pragma unroll
-    for (int i = 1; i < 128; ++i) mx = fmaxf(mx, f[i]);
+    const float mx = fmaxf(max64(f), max64(f + 64));
     // Lazy rescale: keep the stale maximum unless it grew by more than 2^8
     // (P then stays <= 256); the decision is warp-uniform because the O
     // rescale uses warp-collective TMEM loads/stores.
@@ -257,25 +390,13 @@ __device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, const CU
       rescale = true;
     }
     const float neg = -m_used * c;
-    float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2_approx(fmaf(f[64 * h + 2 * i], c, neg));
-        const float p1 = ex2_approx(fmaf(f[64 * h + 2 * i + 1], c, neg));
-        pk[i] = pack_f16(p0, p1);
-        // l sums the fp16-rounded P the MMA multiplies V with, so a row
-        // dominated by one key returns that key's V row exactly
-        if (i & 1)
-          sum1 = add_f16x2_to_f32(sum1, pk[i]);
-        else
-          sum0 = add_f16x2_to_f32(sum0, pk[i]);
-      }
-      tmem_st32(tS + 32 * h, pk);
-    }
-    l += sum0 + sum1;
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t pk[32];
+    exp_half(f, c, neg, pk, sum);
+    tmem_st32(tS, pk);
+    exp_half(f + 64, c, neg, pk, sum);
+    tmem_st32(tS + 32, pk);
+    l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     if (rescale) {
       // O_t holds P V up to tile j-1 (that MMA completed before S_t of
       // tile j was committed) and no MMA writes it until p_ready.
@@ -292,15 +413,15 @@ __device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, const CU
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.p_ready[t]);
+    if (lane == 0) mbar_arrive_remote(p_ready_even);
   }
   // epilogue: O / l and the log-sum-exp
   if (ok && warp_wait(&sm.o_final[t], 0, wc)) {
     tc_fence_after();
-    const int n = q0 + t * kTile + row;
+    const int n = pr.row0[t] + row;
     const bool valid = n < p.N;
     const float inv_l = 1.0f / l;
-    const size_t row_off = (static_cast<size_t>(bh) * p.N + n) * kHeadDim;
+    const size_t row_off = (static_cast<size_t>(pr.bh) * p.N + n) * kHeadDim;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t o[32];
@@ -318,47 +439,60 @@ __device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, const CU
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float* v8 = reinterpret_cast<const float*>(o + 8 * i);
-            dst[i] = make_uint4(pack_bf16(v8[0] * inv_l, v8[1] * inv_l), pack_bf16(v8[2] * inv_l, v8[3] * inv_l),
-                                pack_bf16(v8[4] * inv_l, v8[5] * inv_l), pack_bf16(v8[6] * inv_l, v8[7] * inv_l));
+            dst[i] = make_uint4(pack_bf16x2_rn(v8[0] * inv_l, v8[1] * inv_l),
+                                pack_bf16x2_rn(v8[2] * inv_l, v8[3] * inv_l),
+                                pack_bf16x2_rn(v8[4] * inv_l, v8[5] * inv_l),
+                                pack_bf16x2_rn(v8[6] * inv_l, v8[7] * inv_l));
           }
         }
       }
     }
     if (valid && p.lse != nullptr) {
-      p.lse[static_cast<size_t>(bh) * p.N + n] = (m_used * c + lg2_approx(l)) * 0.69314718055994530942f;
+      p.lse[static_cast<size_t>(pr.bh) * p.N + n] = (m_used * c + lg2_approx(l)) * 0.69314718055994530942f;
     }
   }
 }
 
-// Operand prologue: rotary embedding of Q / K, fp16 conversion of V (warps 2-3, 12-15).
-__device__ __forceinline__ void prologue_role(Smem& sm, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v, uint32_t tmem, int bh, int q0, int warp, int lane, const WaitCtx& wc) {
+// ---------------------------------------------------------------- operand work
+// Rotary embedding of the CTA's two Q tiles by warps 2-15, then one arrive on
+// the even CTA's q_ready.  kBatch: loads in flight per thread.
+template <int kBatch>
+__device__ __forceinline__ void rotate_q(Smem& sm, const Params& p, const Pair& pr, int warp, int lane,
+                                         const WaitCtx& wc) {
+  const int qt = (warp - 2) * 32 + lane;      // 0..447
+  const bool ok = warp_wait(&sm.q_full, 0, wc);
+  if (ok && p.cos != nullptr) {
+    rotate_chunks<kQTileBytes / 16, kQRotThreads, kBatch, false>(sm.q[0], pr.row0[0], p, qt);
+    rotate_chunks<kQTileBytes / 16, kQRotThreads, kBatch, false>(sm.q[1], pr.row0[1], p, qt);
+  }
+  fence_proxy_async_smem();
+  named_bar_sync(kBarQRot, kQRotThreads);
+  if (ok && qt == 0) mbar_arrive_cluster(cl(&sm.q_ready, 0));
+}
+
+// In-loop operand work (warps 2-3, 12-15) on this CTA's K_j and V_j halves.
+__device__ __forceinline__ void kv_prologue_role(Smem& sm, const Params& p, const Pair& pr, int warp, int lane,
+                                                 const WaitCtx& wc) {
   const int pt = (warp < 4 ? (warp - 2) * 32 : 64 + (warp - 12) * 32) + lane;
-  const bool rope = p.cos != nullptr;
-  if (warp_wait(&sm.q_full, 0, wc)) {
-    if (rope) {
-      rotate_tile(sm.q[0], q0, p, pt);
-      rotate_tile(sm.q[1], q0 + kTile, p, pt);
-    }
+  for (int j = 0; j < p.n_kv; ++j) {
+    const int s = j % kStages;
+    const uint32_t ph = (j / kStages) & 1;
+    if (!warp_wait(&sm.k_full[s], ph, wc)) break;
+    if (p.rotate_k)
+      rotate_chunks<kKHalfBytes / 16, kProThreads, 2, true>(sm.k[s], j * kTile + 64 * static_cast<int>(pr.rank),
+                                                            p, pt);
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.q_ready);
-    for (int j = 0; j < p.n_kv; ++j) {
-      const int s = j % kStages;
-      const uint32_t ph = (j / kStages) & 1;
-      if (!warp_wait(&sm.k_full[s], ph, wc)) break;
-      if (rope && p.rotate_k) rotate_tile(sm.k[s], j * kTile, p, pt);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.k_ready[s]);
-      if (!warp_wait(&sm.v_full[s], ph, wc)) break;
-      convert_tile_f16(sm.v[s], pt);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.v_ready[s]);
-    }
+    if (lane == 0) mbar_arrive_cluster(cl(&sm.k_ready[s], 0));
+    if (!warp_wait(&sm.v_full[s], ph, wc)) break;
+    if (p.convert_v) convert_half_f16(sm.v[s], pt);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(cl(&sm.v_ready[s], 0));
   }
 }
 
+template <bool kPrepared>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -366,24 +500,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / p.pairs;
-  const int q0 = (blockIdx.x % p.pairs) * 2 * kTile;
-  const WaitCtx wc{&sm.abort, p.status};
+  Pair pr;
+  pr.rank = cluster_ctarank();
+  pr.peer = pr.rank ^ 1u;
+  const int cluster = blockIdx.x >> 1;
+  pr.bh = cluster / p.clusters;
+  const int q0 = (cluster % p.clusters) * 4 * kTile;
+  pr.row0[0] = q0 + kTile * static_cast<int>(pr.rank);
+  pr.row0[1] = q0 + 2 * kTile + kTile * static_cast<int>(pr.rank);
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_ready, kProWarps);
+    mbar_init(&sm.q_ready, 2);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_ready[s], kProWarps);
+      mbar_init(&sm.k_ready[s], 2 * kProWarps);
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.v_ready[s], kProWarps);
+      mbar_init(&sm.v_ready[s], 2 * kProWarps);
       mbar_init(&sm.v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);
-      mbar_init(&sm.p_ready[t], 4);
+      mbar_init(&sm.p_ready[t], 8);
       mbar_init(&sm.o_final[t], 1);
     }
     mbar_init(&sm.mma_drain, 1);
@@ -391,49 +530,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(&sm.tmem_base, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();          // both CTAs' barriers initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort, p.status, cl(&sm.abort, pr.peer)};
 
-  // 4 warpgroups share 4 x 128 x 128 registers: the two softmax warpgroups
-  // take 192 per thread, the producer / MMA / prologue warpgroups keep 64.
   const int wg = warp >> 2;
   if (wg == 1 || wg == 2) {
-    regs_increase<192>();
-    softmax_role(sm, p, &tm_q, &tm_k, &tm_v, tmem, bh, q0, warp, lane, wc);
+    regs_increase<kSoftmaxRegs>();
+    rotate_q<4>(sm, p, pr, warp, lane, wc);
+    softmax_role(sm, p, tmem, pr, warp, lane, wc);
   } else {
-    regs_decrease<64>();
-    if (warp == 0)
-      producer_role(sm, p, &tm_q, &tm_k, &tm_v, tmem, bh, q0, warp, lane, wc);
-    else if (warp == 1)
-      mma_role(sm, p, &tm_q, &tm_k, &tm_v, tmem, bh, q0, warp, lane, wc);
+    if (wg == 0)
+      regs_decrease<kIssueRegs>();
     else
-      prologue_role(sm, p, &tm_q, &tm_k, &tm_v, tmem, bh, q0, warp, lane, wc);
+      regs_decrease<kOperandRegs>();
+    if (warp == 0) {
+      if (lane == 0) producer_role<kPrepared>(sm, p, &tm_q, &tm_k, &tm_v, pr, wc);
+    } else if (warp == 1) {
+      if (lane == 0 && pr.rank == 0) mma_role<kPrepared>(sm, p, tmem, wc);
+    } else {
+      rotate_q<2>(sm, p, pr, warp, lane, wc);
+      if (!kPrepared) kv_prologue_role(sm, p, pr, warp, lane, wc);
+    }
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();          // no CTA leaves while its peer may still signal it
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
-bool make_map(CUtensorMap* map, const void* base, int BH, int N) {
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, bool f16, int box_rows) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
                                  static_cast<cuuint64_t>(N) * kHeadDim * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   EncodeTiledFn enc = encode_tiled_fn();
   if (enc == nullptr) return false;
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+template <bool kPrepared>
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, long long grid,
+           cudaStream_t s) {
+  const size_t smem = sizeof(Smem) + 1024;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -4;
+  if (configured_device != dev) {
+    if (cudaFuncSetAttribute(attn_fwd_bf16_kernel<kPrepared>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -4;
+    configured_device = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<kPrepared>, mq, mk, mv, p) == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace
@@ -441,7 +615,9 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N) {
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   const int BH = a.B * a.H;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, BH, a.N) || !make_map(&mk, a.k, BH, a.N) || !make_map(&mv, a.v, BH, a.N)) return -4;
+  if (!make_map(&mq, a.q, BH, a.N, false, kTile) || !make_map(&mk, a.k, BH, a.N, false, 64) ||
+      !make_map(&mv, a.v, BH, a.N, a.v_f16, kTile))
+    return -4;
   Params p;
   p.cos = a.cos;
   p.sin = a.sin;
@@ -450,26 +626,16 @@ int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   p.status = device_status_word();
   if (p.status == nullptr) return -4;
   p.N = a.N;
-  p.n_qtiles = (a.N + kTile - 1) / kTile;
-  p.n_kv = p.n_qtiles;
-  p.pairs = (p.n_qtiles + 1) / 2;
+  p.n_kv = (a.N + kTile - 1) / kTile;
+  p.clusters = (a.N + 4 * kTile - 1) / (4 * kTile);
   p.out_f32 = a.out_f32 ? 1 : 0;
   p.rotate_k = (a.cos != nullptr && !a.k_rotated) ? 1 : 0;
+  p.convert_v = a.v_f16 ? 0 : 1;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kHeadDim));
-  const size_t smem = sizeof(Smem) + 1024;
-  static thread_local int configured_device = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -4;
-  if (configured_device != dev) {
-    if (cudaFuncSetAttribute(attn_fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return -4;
-    configured_device = dev;
-  }
-  const long long grid = static_cast<long long>(BH) * p.pairs;
+  const long long grid = 2LL * BH * p.clusters;
   if (grid > 0x7FFFFFFFLL) return -1;
-  attn_fwd_bf16_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  if (!p.rotate_k && !p.convert_v) return launch<true>(mq, mk, mv, p, grid, s);
+  return launch<false>(mq, mk, mv, p, grid, s);
 }
 
 }  // namespace dit

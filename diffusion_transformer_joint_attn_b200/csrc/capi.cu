@@ -78,6 +78,21 @@ int dit_rope_apply(const void* x, const float* rope_cos, const float* rope_sin, 
   return dit::launch_rope_apply(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
+int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, const float* rope_sin, void* k_rot,
+                        void* v_f16, int B, int H, int N, int D, dit_stream_t stream) {
+  if (k == nullptr || v == nullptr || rope_cos == nullptr || rope_sin == nullptr || k_rot == nullptr ||
+      v_f16 == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * N > (1LL << 40)) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_rot) || !aligned16(v_f16) || !aligned16(rope_cos) ||
+      !aligned16(rope_sin))
+    return DIT_ERR_MISALIGNED;
+  dit::PrepareKVArgs a{k, v, rope_cos, rope_sin, k_rot, v_f16, B, H, N, D};
+  return dit::launch_prepare_kv(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                      void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
                      dit_stream_t stream) {
@@ -88,13 +103,13 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
   if (N < 1 || N > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
   if (D != 128) return DIT_ERR_UNSUPPORTED;
-  if ((dtype & ~(DIT_OUT_F32 | DIT_K_ROTATED)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+  if ((dtype & ~(DIT_OUT_F32 | DIT_K_ROTATED | DIT_V_F16)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
   if ((dtype & DIT_K_ROTATED) && rope_cos == nullptr) return DIT_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIT_ERR_MISALIGNED;
   if ((rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) || (lse != nullptr && !aligned4(lse)))
     return DIT_ERR_MISALIGNED;
   dit::AttnFwdArgs a{q,   k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N), (dtype & DIT_OUT_F32) != 0,
-                     (dtype & DIT_K_ROTATED) != 0};
+                     (dtype & DIT_K_ROTATED) != 0, (dtype & DIT_V_F16) != 0};
   return dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -30,6 +30,17 @@ struct RopeApplyArgs {
 };
 cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t s);
 
+struct PrepareKVArgs {
+  const void* k;
+  const void* v;
+  const float* cos;
+  const float* sin;
+  void* k_rot;     // bf16, rotated
+  void* v_f16;     // fp16 copy of v
+  int B, H, N, D;
+};
+cudaError_t launch_prepare_kv(const PrepareKVArgs& a, cudaStream_t s);
+
 struct AttnFwdArgs {
   const void* q;
   const void* k;
@@ -41,6 +52,7 @@ struct AttnFwdArgs {
   int B, H, N;
   bool out_f32;
   bool k_rotated;   // k already carries the rotary embedding: rotate q only
+  bool v_f16;       // v is given as fp16 (otherwise bf16)
 };
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.

@@ -56,6 +56,7 @@ typedef enum {
 typedef enum { DIT_BF16 = 0, DIT_FP8_E4M3 = 1 } dit_dtype_t;
 #define DIT_OUT_F32 0x100   /* write `out` as fp32 instead of bf16 */
 #define DIT_K_ROTATED 0x200 /* k already carries the rotary embedding (dit_rope_apply); rotate q only */
+#define DIT_V_F16 0x400     /* v is given as fp16 (dit_attn_prepare_kv) instead of bf16 */
 
 /*
  * dit_rope_table_build — cos/sin table of the three-axis rotary embedding.
@@ -99,6 +100,25 @@ int dit_rope_apply(const void* x, const float* rope_cos, const float* rope_sin, 
                    int D, dit_stream_t stream);
 
 /*
+ * dit_attn_prepare_kv — the operands of the attention's two products,
+ * prepared once per call in one memory-bound pass:
+ *
+ *   k, v      device bf16 [B][H][N][D].
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2] from dit_rope_table_build.
+ *   k_rot     device bf16 [B][H][N][D], written: k rotated exactly as by
+ *             dit_rope_apply.
+ *   v_f16     device fp16 [B][H][N][D], written: v converted to fp16 (exact for
+ *             2^-14 <= |v| <= 65504; |v| > 65504 is outside the contract).
+ *   B, H, N   >= 1;  D must be 128.  All pointers 16-byte aligned.
+ * dit_attn_forward(q, k_rot, v_f16, ..., DIT_K_ROTATED | DIT_V_F16) returns bit
+ * for bit what dit_attn_forward(q, k, v, ...) does, and is the fast path: the
+ * attention kernel then does no per-tile operand work for K and V.
+ */
+int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, const float* rope_sin, void* k_rot,
+                        void* v_f16, int B, int H, int N, int D, dit_stream_t stream);
+
+/*
  * dit_attn_forward — joint attention forward, BF16 in, BF16 (or fp32) out.
  *
  *   q, k, v   device bf16 [B][H][N][D], N = N_txt + N_img.
@@ -115,8 +135,9 @@ int dit_rope_apply(const void* x, const float* rope_cos, const float* rope_sin, 
  *             token attends to all N tokens (no mask); positions enter only
  *             through the tables.
  *   D         head dimension; must be 128.
- *   dtype     DIT_BF16, optionally | DIT_OUT_F32 and | DIT_K_ROTATED (the
- *             latter requires the tables: they are then applied to q only).
+ *   dtype     DIT_BF16, optionally | DIT_OUT_F32, | DIT_K_ROTATED (requires
+ *             the tables: they are then applied to q only) and | DIT_V_F16
+ *             (v holds fp16 values, as written by dit_attn_prepare_kv).
  *
  * Precision: each rotated component of q and k is the bf16 nearest to its
  * exact value for the fp32 table entries; q~ k~^T accumulates in fp32; the

@@ -40,12 +40,21 @@ def errors(got, ref):
     return float(e.max()), float(e.mean())
 
 
-def run_gpu(w, rope=True, out_f32=False, seed=0, inputs=None):
+def run_gpu(w, rope=True, out_f32=False, seed=0, inputs=None, prepared=True):
+    """prepared: K / V go through dit_attn_prepare_kv first (the fast path);
+    otherwise the kernel rotates K and converts V tile by tile."""
     if inputs is None:
         inputs = device_inputs(w, seed)
     q, k, v, qd, kd, vd = inputs
     cs = rope_tables(w) if rope else (None, None)
-    out, lse = dit.forward(qd, kd, vd, cs[0], cs[1], n_txt=w.n_txt, out_f32=out_f32)
+    if prepared and rope:
+        kr = torch.empty_like(kd)
+        v16 = torch.empty(vd.shape, dtype=torch.float16, device=vd.device)
+        dit.dit_attn_prepare_kv(kd, vd, cs[0], cs[1], kr, v16)
+        out, lse = dit.forward(qd, kr, v16, cs[0], cs[1], n_txt=w.n_txt, out_f32=out_f32, k_rotated=True,
+                               v_f16=True)
+    else:
+        out, lse = dit.forward(qd, kd, vd, cs[0], cs[1], n_txt=w.n_txt, out_f32=out_f32)
     torch.cuda.synchronize()
     assert dit.dit_attn_get_status() == dit.DIT_OK
     return out, lse

@@ -60,7 +60,8 @@ def test_forward_argument_errors(lib):
     assert _fwd(lib, nt=2 ** 31 - 1, ni=2) == dit.DIT_ERR_INVALID_ARG
     assert _fwd(lib, D=64) == dit.DIT_ERR_UNSUPPORTED
     assert _fwd(lib, dtype=dit.DIT_FP8_E4M3) == dit.DIT_ERR_UNSUPPORTED
-    assert _fwd(lib, dtype=0x400) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=0x800) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=dit.DIT_K_ROTATED) == dit.DIT_ERR_INVALID_ARG      # flag without tables
     assert _fwd(lib, q=0x10008) == dit.DIT_ERR_MISALIGNED
     assert _fwd(lib, out=0x40004) == dit.DIT_ERR_MISALIGNED
     assert _fwd(lib, cos=0x50000, sin=0x60008) == dit.DIT_ERR_MISALIGNED
@@ -80,6 +81,24 @@ def test_rope_table_argument_errors(lib):
     assert f(0x100, 8, 96, ax, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_UNSUPPORTED
     assert f(0x102, 8, 128, ax, 1e4, 0x1000, 0x2000, None) == dit.DIT_ERR_MISALIGNED
     assert f(0x100, 8, 128, ax, 1e4, 0x1004, 0x2000, None) == dit.DIT_ERR_MISALIGNED
+
+
+def test_operand_pass_argument_errors(lib):
+    f = lib.dit_attn_prepare_kv
+    ok = dict(k=0x1000, v=0x2000, c=0x3000, s=0x4000, kr=0x5000, vf=0x6000, B=1, H=1, N=8, D=128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["k"], a["v"], a["c"], a["s"], a["kr"], a["vf"], a["B"], a["H"], a["N"], a["D"], None)
+    assert call(k=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(vf=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(N=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(v=0x2008) == dit.DIT_ERR_MISALIGNED
+    g = lib.dit_rope_apply
+    assert g(None, 0x3000, 0x4000, 0x5000, 1, 1, 8, 128, None) == dit.DIT_ERR_INVALID_ARG
+    assert g(0x1000, 0x3000, 0x4000, 0x5000, 1, 1, 8, 64, None) == dit.DIT_ERR_UNSUPPORTED
+    assert g(0x1004, 0x3000, 0x4000, 0x5000, 1, 1, 8, 128, None) == dit.DIT_ERR_MISALIGNED
 
 
 def test_get_status_rejects_null(lib):

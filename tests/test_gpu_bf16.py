@@ -105,8 +105,8 @@ def test_parity_ragged_shapes(B, H, n_txt, grids):
     q, k, v = inputs[:3]
     rows = W.sample_rows(w)
     O_ref, L_ref = oracle_rows(w, q, k, v, rows)
-    out, lse = run_gpu(w, inputs=inputs)
-    check(out, lse, rows, O_ref, L_ref, "ragged N=%d bf16-out" % w.N, gate_lse=False)
+    out, lse = run_gpu(w, inputs=inputs, prepared=False)
+    check(out, lse, rows, O_ref, L_ref, "ragged N=%d bf16-out (fused)" % w.N, gate_lse=False)
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
     O_op, L_op = oracle_rows(w, q, k, v, rows, operands="bf16")
     check(out32, lse32, rows, O_op, L_op, "ragged N=%d fp32-out" % w.N)
@@ -140,7 +140,7 @@ def test_rope_apply_is_exactly_rounded():
 
 
 @pytest.mark.parametrize("name", ["tiny_256", "t2i_2048px"])
-def test_prerotated_k_matches_fused_rotation_bitwise(name):
+def test_prepared_operands_match_fused_path_bitwise(name):
     w = W.WORKLOADS[name]
     _, _, _, qd, kd, vd = device_inputs(w)
     c, s = dit.rope_table(torch.from_numpy(W.positions(w)).cuda())
@@ -148,8 +148,14 @@ def test_prerotated_k_matches_fused_rotation_bitwise(name):
     kr = torch.empty_like(kd)
     dit.dit_rope_apply(kd, c, s, kr)
     b, lb = dit.forward(qd, kr, vd, c, s, n_txt=w.n_txt, k_rotated=True)
+    kr2 = torch.empty_like(kd)
+    v16 = torch.empty(vd.shape, dtype=torch.float16, device=vd.device)
+    dit.dit_attn_prepare_kv(kd, vd, c, s, kr2, v16)
+    d, ld = dit.forward(qd, kr2, v16, c, s, n_txt=w.n_txt, k_rotated=True, v_f16=True)
     torch.cuda.synchronize()
+    assert torch.equal(kr, kr2) and torch.equal(v16, vd.to(torch.float16))
     assert torch.equal(a, b) and torch.equal(la, lb)
+    assert torch.equal(a, d) and torch.equal(la, ld)
 
 
 def test_lse_may_be_omitted():
