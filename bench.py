@@ -146,9 +146,9 @@ def measured_peaks():
     return FALLBACK_PEAK_BF16, "fallback 1.59 PFLOP/s"
 
 
-def profile_traffic(kernel_source_sha: str):
-    """DRAM bytes per launch of the attention kernel from the committed ncu
-    summary, or None if none exists for the current kernel source."""
+def profile_traffic(kernel_source_sha: str, kernel: str):
+    """DRAM bytes per launch of `kernel` on the bench workload from the
+    committed ncu summary, or None if none exists for the current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -156,7 +156,7 @@ def profile_traffic(kernel_source_sha: str):
         d = json.load(f)
     if d.get("source_sha") != kernel_source_sha or d.get("workload") != WORKLOAD:
         return None
-    return d.get("dram_bytes_per_launch")
+    return d.get("kernels", {}).get(kernel, {}).get("dram_bytes_per_launch")
 
 
 def kernel_source_sha() -> str:
@@ -185,6 +185,67 @@ def time_oracle(w, q, k, v, rows):
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     flops = 4.0 * w.N * w.D * len(rows)
     return flops / dt / 1e12, dt, threads
+
+
+def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, world):
+    """The FP8 E4M3 variant on the same inputs: per-64-token quantisation of
+    the rotated q, k and of v, then the FP8 attention forward.  Timed apart
+    from the BF16 step; the kernel's roofline peak mixes the two tensor rates
+    (q k^T on E4M3 operands at twice the bf16 rate, P V in fp16)."""
+    import torch
+    import diffusion_transformer_joint_attn_b200 as dit
+    nb = (w.N + 63) // 64
+    q8, k8, v8 = (torch.empty(q.shape, dtype=torch.uint8, device=dev) for _ in range(3))
+    qs, ks, vs = (torch.empty((w.B, w.H, nb), dtype=torch.float32, device=dev) for _ in range(3))
+    s_ptr = stream.cuda_stream
+
+    def step(ev=None):
+        assert lib.dit_attn_quantize_fp8(q.data_ptr(), cos.data_ptr(), sin.data_ptr(), q8.data_ptr(), qs.data_ptr(),
+                                         w.B, w.H, w.N, w.D, s_ptr) == 0
+        assert lib.dit_attn_quantize_fp8(k.data_ptr(), cos.data_ptr(), sin.data_ptr(), k8.data_ptr(), ks.data_ptr(),
+                                         w.B, w.H, w.N, w.D, s_ptr) == 0
+        assert lib.dit_attn_quantize_fp8(v.data_ptr(), None, None, v8.data_ptr(), vs.data_ptr(),
+                                         w.B, w.H, w.N, w.D, s_ptr) == 0
+        if ev is not None:
+            ev[0].record(stream)
+        assert lib.dit_attn_forward_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), qs.data_ptr(), ks.data_ptr(),
+                                        vs.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B, w.H, w.n_txt, w.n_img,
+                                        w.D, dit.DIT_FP8_E4M3, s_ptr) == 0
+        if ev is not None:
+            ev[1].record(stream)
+
+    steps = max(1, min(args.steps, 50))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    kern_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(steps):
+        step(kern_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dit.dit_attn_get_status(stream) != 0:
+        raise RuntimeError("device status error in the FP8 timed region")
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    kern_ms = sum(a.elapsed_time(b) for a, b in kern_ev) / steps
+    peak_bf16, src = measured_peaks()
+    # minimum time = (F/2) / (2 P) + (F/2) / P = 0.75 F / P
+    peak = peak_bf16 / 0.75
+    achieved = w.flops / (kern_ms * 1e-3) / 1e12
+    return {"value": whole_job_throughput(w.flops, steps, world, max_ms), "unit": UNIT, "steps": steps,
+            "ms_per_step": max_ms / steps, "dtype": "e4m3 (q k^T), fp16 (P V)",
+            "step": "quantise rotated q, k and v to E4M3 (per 64 tokens) + FP8 attention forward",
+            "gpu_launches": 4 * steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "kernel": "attn_fwd_fp8_kernel",
+                         "traffic": profile_traffic(kernel_source_sha(), "attn_fwd_fp8_kernel")
+                         if w.name == WORKLOAD else None,
+                         "peak_source": src + " x 4/3 (q k^T at the nominal 2x E4M3 rate, P V at the bf16 rate)",
+                         "kernel_ms": kern_ms}}
 
 
 # ------------------------------------------------------------------ native arm
@@ -256,6 +317,8 @@ def run_native(args):
     max_ms = max_over_ranks(ms, world, dev)
     value = whole_job_throughput(w.flops, args.steps, world, max_ms)
 
+    fp8 = time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, world)
+
     # end to end through the public API: pinned host inputs in, O and LSE out
     q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     pos_p = pos_h.pin_memory()
@@ -290,7 +353,7 @@ def run_native(args):
 
     peak, peak_src = measured_peaks()
     achieved = w.flops / (kern_ms * 1e-3) / 1e12
-    traffic = profile_traffic(kernel_source_sha()) if w.name == WORKLOAD else None
+    traffic = profile_traffic(kernel_source_sha(), "attn_fwd_bf16_kernel") if w.name == WORKLOAD else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -318,6 +381,7 @@ def run_native(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": 3 * args.steps,
+            "fp8": fp8,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }

@@ -122,6 +122,57 @@ def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: i
            "dit_attn_forward")
 
 
+def dit_attn_quantize_fp8(x, rope_cos, rope_sin, x_fp8, scale, stream=None) -> None:
+    """x_fp8 (uint8 E4M3 codes) and scale (fp32 per 64-token block) of bf16 x [B, H, N, D]."""
+    import torch
+    _require(x.dim() == 4 and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous(), "x must be CUDA bf16")
+    B, H, N, D = x.shape
+    _require(x_fp8.is_cuda and x_fp8.dtype == torch.uint8 and x_fp8.is_contiguous() and x_fp8.shape == x.shape,
+             "x_fp8 must be a contiguous CUDA uint8 tensor of x's shape")
+    _require(scale.is_cuda and scale.dtype == torch.float32 and scale.is_contiguous() and
+             tuple(scale.shape) == (B, H, (N + 63) // 64), "scale must be CUDA fp32 [B, H, ceil(N/64)]")
+    if rope_cos is not None or rope_sin is not None:
+        for t in (rope_cos, rope_sin):
+            _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _check(load_library().dit_attn_quantize_fp8(_ptr(x), _ptr(rope_cos), _ptr(rope_sin), _ptr(x_fp8), _ptr(scale),
+                                                B, H, N, D, _stream(stream)), "dit_attn_quantize_fp8")
+
+
+def quantize_fp8(x, rope_cos=None, rope_sin=None, stream=None):
+    """Allocate and fill (codes, scales) for bf16 x [B, H, N, D]."""
+    import torch
+    B, H, N, D = x.shape
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = torch.empty((B, H, (N + 63) // 64), dtype=torch.float32, device=x.device)
+    dit_attn_quantize_fp8(x, rope_cos, rope_sin, codes, scale, stream)
+    return codes, scale
+
+
+def dit_attn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, n_txt: int, n_img: int,
+                         dtype: int = DIT_FP8_E4M3, stream=None) -> None:
+    """out (and lse, if not None) <- joint attention of E4M3 codes q8, k8, v8 [B, H, N, D] with
+    per-64-token fp32 scales [B, H, ceil(N/64)]."""
+    import torch
+    _require(q8.dim() == 4 and q8.shape == k8.shape == v8.shape, "q8, k8, v8 must share one [B, H, N, D] shape")
+    B, H, N, D = q8.shape
+    _require(N == n_txt + n_img, "N must equal n_txt + n_img")
+    for t in (q8, k8, v8):
+        _require(t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous(), "q8, k8, v8 must be contiguous CUDA uint8")
+    for t in (q_scale, k_scale, v_scale):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                 tuple(t.shape) == (B, H, (N + 63) // 64), "scales must be contiguous CUDA fp32 [B, H, ceil(N/64)]")
+    out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
+    _require(out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q8.shape,
+             "out must be a contiguous CUDA tensor of q8's shape and the requested dtype")
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, N),
+                 "lse must be a contiguous CUDA fp32 [B, H, N] tensor")
+    _check(load_library().dit_attn_forward_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale),
+                                               _ptr(v_scale), _ptr(out), _ptr(lse), B, H, n_txt, n_img, D, dtype,
+                                               _stream(stream)), "dit_attn_forward_fp8")
+
+
 def dit_attn_get_status(stream=None) -> int:
     """Synchronise the stream, return and clear the device status word."""
     st = ctypes.c_int(0)
@@ -153,4 +204,16 @@ def forward(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
     flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0) | (DIT_V_F16 if v_f16 else 0)
     dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt, DIT_BF16 | flags, stream)
+    return out, lse
+
+
+def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, n_txt: int = 0, out_f32: bool = False,
+                with_lse: bool = True, stream=None):
+    """Allocate out (and lse) and run dit_attn_forward_fp8; returns (out, lse)."""
+    import torch
+    B, H, N, D = q8.shape
+    out = torch.empty(q8.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device) if with_lse else None
+    dit_attn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, n_txt, N - n_txt,
+                         DIT_FP8_E4M3 | (DIT_OUT_F32 if out_f32 else 0), stream)
     return out, lse

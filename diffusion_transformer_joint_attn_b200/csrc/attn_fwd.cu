@@ -27,16 +27,19 @@
 // fp32 columns each; P_t (fp16) overwrites the first 64 columns of S_t.
 // While the softmax warps of one slot work, the tensor cores run the other
 // slot's MMAs.
+#include "attn_common.cuh"
 #include "launch.h"
-#include "ptx.cuh"
-#include "rope_exact.cuh"
-#include "softmax_exp2.cuh"
 
 namespace dit {
 namespace {
 
-constexpr int kTile = 128;                         // query rows per tile = keys per K/V tile
-constexpr int kHeadDim = 128;
+using attn::cl;
+using attn::commit_both;
+using attn::kHeadDim;
+using attn::kTile;
+using attn::pack_f16;
+using attn::Pair;
+
 constexpr int kStages = 4;                         // K and V ring depth
 constexpr int kQTileBytes = kTile * kHeadDim * 2;  // 32 KB: 128 rows x 128 channels
 constexpr int kQBoxBytes = kTile * 64 * 2;         // 16 KB: 128 rows x 64 channels
@@ -48,7 +51,6 @@ constexpr int kProWarps = 6;                       // in-loop operand warps per 
 constexpr int kProThreads = kProWarps * 32;
 constexpr int kQRotThreads = 14 * 32;              // warps 2-15 rotate Q
 constexpr int kBarQRot = 1;                        // named barrier of the Q rotation
-constexpr int kPolyEvery = 4;                      // every kPolyEvery-th exponent pair on the FMA pipe (0: none)
 // Register split of the 4 x 128 x 128 launch registers between warpgroups:
 // producer / MMA warpgroup, the two softmax warpgroups, the operand warpgroup.
 constexpr uint32_t kIssueRegs = 80;
@@ -85,16 +87,6 @@ struct Params {
   float scale_log2;   // log2(e) / sqrt(D)
 };
 
-struct Pair {
-  uint32_t rank;      // 0: even (MMA-issuing) CTA, 1: odd CTA
-  uint32_t peer;
-  int bh;
-  int row0[2];        // first query row of this CTA's tile in slot 0 / 1
-};
-
-// shared::cluster address of `p` in CTA `rank` of the pair.
-__device__ __forceinline__ uint32_t cl(const void* p, uint32_t rank) { return mapa_shared(smem_u32(p), rank); }
-
 // Q tile chunk c (0..2047): byte offset in the 128B-swizzled layout of two
 // 128-row x 64-channel boxes, its row and first channel.
 __device__ __forceinline__ void q_chunk(int c, int& byte_off, int& row, int& col0) {
@@ -115,10 +107,6 @@ __device__ __forceinline__ void k_chunk(int c, int& byte_off, int& row, int& col
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 // Rotate chunks first, first+kStep, ... (< kChunks) of a tile whose row r is
 // token n0 + r, in place, each component rounded exactly to bf16.  The loads
@@ -242,11 +230,6 @@ __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const C
 // ---------------------------------------------------------------- MMA issuer
 // Even CTA only.  Completion of pair MMAs is signalled to the barrier of the
 // same name in both CTAs.
-__device__ __forceinline__ void commit_both(uint64_t* bar) {
-  tc_commit_pair(cl(bar, 0));
-  tc_commit_pair(cl(bar, 1));
-}
-
 template <bool kPrepared>
 __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tmem, const WaitCtx& wc) {
   constexpr uint32_t idesc_qk = instr_desc(1, 1, 256, 128, 0, 0);   // bf16 x bf16, both K-major
@@ -304,153 +287,6 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
   // every MMA issued above has completed once this arrives
   tc_commit_pair(cl(&sm.mma_drain, 0));
   mbar_wait_drain(&sm.mma_drain, 0, wc);
-}
-
-// ---------------------------------------------------------------- softmax
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// Max of 64 consecutive values (4 independent chains of 3-input max).
-__device__ __forceinline__ float max64(const float* f) {
-  float m[4] = {f[0], f[1], f[2], f[3]};
-#pragma unroll
-  for (int i = 4; i < 64; i += 8) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) m[u] = fmax3(m[u], f[i + 2 * u], f[i + 2 * u + 1]);
-  }
-  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-}
-
-// P for 64 consecutive logits of the row: 2^(s c - m c) rounded to fp16, packed
-// in pairs into pk[32]; adds the rounded values to sum[4].
-__device__ __forceinline__ void exp_half(const float* f, float c, float neg, uint32_t* pk, float* sum) {
-  const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float2 x = __ffma2_rn(make_float2(f[2 * i], f[2 * i + 1]), c2, n2);
-    float e0, e1;
-    if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
-      exp2_pair_poly(x.x, x.y, e0, e1);
-    } else {
-      e0 = ex2_approx(x.x);
-      e1 = ex2_approx(x.y);
-    }
-    pk[i] = pack_f16(e0, e1);
-    // l sums the fp16-rounded P the MMA multiplies V with, so a row
-    // dominated by one key returns that key's V row exactly
-    sum[i & 3] = add_f16x2_to_f32(sum[i & 3], pk[i]);
-  }
-}
-
-// Online softmax and epilogue of this CTA's tile of one slot (warps 4-11).
-__device__ __forceinline__ void softmax_role(Smem& sm, const Params& p, uint32_t tmem, const Pair& pr, int warp,
-                                             int lane, const WaitCtx& wc) {
-  const int t = (warp - 4) >> 2;
-  const int quarter = warp & 3;
-  const int row = quarter * 32 + lane;
-  const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t tS = tmem + lane_base + t * 128;
-  const uint32_t tO = tmem + lane_base + 256 + t * 128;
-  const uint32_t p_ready_even = cl(&sm.p_ready[t], 0);
-  const float c = p.scale_log2;
-  const float rescale_gap = 8.0f / c;     // lazy rescale once the max grew by 2^8
-  const int last_valid = p.N - (p.n_kv - 1) * kTile;
-  float m_used = 0.f, l = 0.f;
-  bool ok = true;
-  for (int j = 0; j < p.n_kv; ++j) {
-    if (!(ok = warp_wait(&sm.s_full[t], j & 1, wc))) break;
-    tc_fence_after();
-    uint32_t s[128];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, s + q * 32);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld_wait(s + q * 32);
-    float* f = reinterpret_cast<float*>(s);
-    if (j == p.n_kv - 1 && last_valid < kTile) {
-#pragma unroll
-      for (int i = 0; i < 128; ++i)
-        if (i >= last_valid) f[i] = -INFINITY;
-    }
-    const float mx = fmaxf(max64(f), max64(f + 64));
-    // Lazy rescale: keep the stale maximum unless it grew by more than 2^8
-    // (P then stays <= 256); the decision is warp-uniform because the O
-    // rescale uses warp-collective TMEM loads/stores.
-    float alpha = 1.0f;
-    bool rescale = false;
-    if (j == 0) {
-      m_used = mx;
-    } else if (__any_sync(0xffffffffu, mx > m_used + rescale_gap)) {
-      const float m_new = fmaxf(m_used, mx);
-      alpha = ex2_approx((m_used - m_new) * c);
-      m_used = m_new;
-      l *= alpha;
-      rescale = true;
-    }
-    const float neg = -m_used * c;
-    float sum[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t pk[32];
-    exp_half(f, c, neg, pk, sum);
-    tmem_st32(tS, pk);
-    exp_half(f + 64, c, neg, pk, sum);
-    tmem_st32(tS + 32, pk);
-    l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
-    if (rescale) {
-      // O_t holds P V up to tile j-1 (that MMA completed before S_t of
-      // tile j was committed) and no MMA writes it until p_ready.
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[32];
-        tmem_ld32(tO + q * 32, o);
-        tmem_ld_wait(o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-        tmem_st32(tO + q * 32, o);
-      }
-    }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_remote(p_ready_even);
-  }
-  // epilogue: O / l and the log-sum-exp
-  if (ok && warp_wait(&sm.o_final[t], 0, wc)) {
-    tc_fence_after();
-    const int n = pr.row0[t] + row;
-    const bool valid = n < p.N;
-    const float inv_l = 1.0f / l;
-    const size_t row_off = (static_cast<size_t>(pr.bh) * p.N + n) * kHeadDim;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t o[32];
-      tmem_ld32(tO + q * 32, o);
-      tmem_ld_wait(o);
-      if (valid) {
-        if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_off + q * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                                 __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_off + q * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float* v8 = reinterpret_cast<const float*>(o + 8 * i);
-            dst[i] = make_uint4(pack_bf16x2_rn(v8[0] * inv_l, v8[1] * inv_l),
-                                pack_bf16x2_rn(v8[2] * inv_l, v8[3] * inv_l),
-                                pack_bf16x2_rn(v8[4] * inv_l, v8[5] * inv_l),
-                                pack_bf16x2_rn(v8[6] * inv_l, v8[7] * inv_l));
-          }
-        }
-      }
-    }
-    if (valid && p.lse != nullptr) {
-      p.lse[static_cast<size_t>(pr.bh) * p.N + n] = (m_used * c + lg2_approx(l)) * 0.69314718055994530942f;
-    }
-  }
 }
 
 // ---------------------------------------------------------------- operand work
@@ -543,7 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (wg == 1 || wg == 2) {
     regs_increase<kSoftmaxRegs>();
     rotate_q<4>(sm, p, pr, warp, lane, wc);
-    softmax_role(sm, p, tmem, pr, warp, lane, wc);
+    attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.n_kv, p.out_f32, p.scale_log2,
+                       nullptr, nullptr, 0};
+    attn::softmax_slot<false>(io, tmem, pr, warp, lane, wc);
   } else {
     if (wg == 0)
       regs_decrease<kIssueRegs>();

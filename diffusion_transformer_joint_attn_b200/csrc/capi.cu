@@ -113,6 +113,38 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
   return dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream));
 }
 
+int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float* rope_sin, uint8_t* x_fp8,
+                          float* scale, int B, int H, int N, int D, dit_stream_t stream) {
+  if (x_bf16 == nullptr || x_fp8 == nullptr || scale == nullptr) return DIT_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * ((N + 63) / 64) > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(x_bf16) || !aligned16(x_fp8) || !aligned4(scale)) return DIT_ERR_MISALIGNED;
+  if (rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) return DIT_ERR_MISALIGNED;
+  dit::QuantFp8Args a{x_bf16, rope_cos, rope_sin, x_fp8, scale, B, H, N};
+  return dit::launch_quantize_fp8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* q_scale,
+                         const float* k_scale, const float* v_scale, void* out, float* lse, int B, int H,
+                         int N_txt, int N_img, int D, int dtype, dit_stream_t stream) {
+  if (q8 == nullptr || k8 == nullptr || v8 == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (q_scale == nullptr || k_scale == nullptr || v_scale == nullptr) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N_txt < 0 || N_img < 0) return DIT_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img;
+  if (N < 1 || N > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if ((dtype & ~DIT_OUT_F32) != DIT_FP8_E4M3) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(out)) return DIT_ERR_MISALIGNED;
+  if (!aligned4(q_scale) || !aligned4(k_scale) || !aligned4(v_scale) || (lse != nullptr && !aligned4(lse)))
+    return DIT_ERR_MISALIGNED;
+  dit::AttnFwdFp8Args a{q8, k8, v8, q_scale, k_scale, v_scale, out, lse, B, H, static_cast<int>(N),
+                        (dtype & DIT_OUT_F32) != 0};
+  return dit::launch_attn_fwd_fp8(a, static_cast<cudaStream_t>(stream));
+}
+
 int dit_attn_get_status(int* status_host, dit_stream_t stream) {
   if (status_host == nullptr) return DIT_ERR_INVALID_ARG;
   int* word = dit::device_status_word();

@@ -41,6 +41,16 @@ struct PrepareKVArgs {
 };
 cudaError_t launch_prepare_kv(const PrepareKVArgs& a, cudaStream_t s);
 
+struct QuantFp8Args {
+  const void* x;       // bf16 [B][H][N][128]
+  const float* cos;    // [N][64] or nullptr (no rotation)
+  const float* sin;
+  void* codes;         // e4m3 [B][H][N][128]
+  float* scale;        // [B][H][ceil(N/64)]
+  int B, H, N;
+};
+cudaError_t launch_quantize_fp8(const QuantFp8Args& a, cudaStream_t s);
+
 struct AttnFwdArgs {
   const void* q;
   const void* k;
@@ -54,6 +64,20 @@ struct AttnFwdArgs {
   bool k_rotated;   // k already carries the rotary embedding: rotate q only
   bool v_f16;       // v is given as fp16 (otherwise bf16)
 };
+struct AttnFwdFp8Args {
+  const void* q8;      // e4m3 [B][H][N][128]
+  const void* k8;
+  const void* v8;
+  const float* q_scale;   // [B][H][ceil(N/64)]
+  const float* k_scale;
+  const float* v_scale;
+  void* out;
+  float* lse;
+  int B, H, N;
+  bool out_f32;
+};
+int launch_attn_fwd_fp8(const AttnFwdFp8Args& a, cudaStream_t s);
+
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s);

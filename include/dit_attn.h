@@ -152,6 +152,54 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
                      dit_stream_t stream);
 
 /*
+ * dit_attn_quantize_fp8 — FP8 E4M3 operands for dit_attn_forward_fp8.
+ *
+ *   x_bf16    device bf16 [B][H][N][D] (q, k or v).
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2]: rotate first (q and k), or both NULL (v).
+ *             Each rotated value x c - y s (or x s + y c) is evaluated in
+ *             fp64 from the fp32 table entries (both products exact, one
+ *             rounding of the sum) and then rounded to fp32.
+ *   x_fp8     device uint8 [B][H][N][D], written: E4M3 ("e4m3fn": bias 7,
+ *             largest finite 448, no infinities) codes.
+ *   scale     device fp32 [B][H][ceil(N/64)], written: one scale per block of
+ *             64 consecutive tokens x all D channels of one (b, h):
+ *             amax / 448 in fp32, or 1 for an all-zero block.
+ *   B, H, N   >= 1;  D must be 128.
+ * Each element's code is the E4M3 value nearest (ties to even) to the fp32
+ * quotient x / scale, saturated to +-448; x = code * scale approximately.
+ * x_bf16, x_fp8 and the tables 16-byte aligned, scale 4-byte aligned.
+ * FP8 attention is prior art on the pages (cuDNN FP8, VC-Attention FP8 on
+ * B200: scopeai.cc, section on each optimisation's effect); the block scheme
+ * is this library's.
+ */
+int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float* rope_sin, uint8_t* x_fp8,
+                          float* scale, int B, int H, int N, int D, dit_stream_t stream);
+
+/*
+ * dit_attn_forward_fp8 — joint attention on FP8 E4M3 operands (dit_attn_quantize_fp8
+ * output; the rotary embedding of q and k was applied before quantisation).
+ *
+ *   q8, k8, v8  device uint8 [B][H][N][D] E4M3 codes, N = N_txt + N_img.
+ *   q_scale, k_scale, v_scale
+ *               device fp32 [B][H][ceil(N/64)]: the value of a code in
+ *               token block n/64 is code * scale.
+ *   out         device [B][H][N][D], bf16, or fp32 when dtype has DIT_OUT_F32.
+ *   lse         device fp32 [B][H][N] or NULL: natural-log sum-exp of the
+ *               scaled logits of each row.
+ *   dtype       DIT_FP8_E4M3, optionally | DIT_OUT_F32.
+ * Computes softmax(q k^T / sqrt(D)) v of the dequantised values: S is formed
+ * from the codes on the 8-bit tensor cores and scaled per (query block, key
+ * block) in fp32; P (fp16) multiplies v dequantised to fp16 (code * scale,
+ * rounded once), accumulating in fp32.  Same limits, alignment (16 bytes for
+ * every pointer, 4 for the scales and lse), status words and asynchrony as
+ * dit_attn_forward.
+ */
+int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* q_scale,
+                         const float* k_scale, const float* v_scale, void* out, float* lse, int B, int H,
+                         int N_txt, int N_img, int D, int dtype, dit_stream_t stream);
+
+/*
  * dit_attn_get_status — synchronise `stream`, copy the device status word to
  * *status_host (DIT_OK or DIT_ERR_TIMEOUT) and reset it to DIT_OK.  Returns
  * DIT_OK, or DIT_ERR_CUDA if the synchronisation or copy failed (for example

@@ -101,6 +101,34 @@ def test_operand_pass_argument_errors(lib):
     assert g(0x1004, 0x3000, 0x4000, 0x5000, 1, 1, 8, 128, None) == dit.DIT_ERR_MISALIGNED
 
 
+def test_fp8_argument_errors(lib):
+    f = lib.dit_attn_quantize_fp8
+    assert f(None, None, None, 0x2000, 0x3000, 1, 1, 8, 128, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x1000, 0x4000, None, 0x2000, 0x3000, 1, 1, 8, 128, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x1000, None, None, 0x2000, 0x3000, 1, 1, 0, 128, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(0x1000, None, None, 0x2000, 0x3000, 1, 1, 8, 64, None) == dit.DIT_ERR_UNSUPPORTED
+    assert f(0x1000, None, None, 0x2008, 0x3000, 1, 1, 8, 128, None) == dit.DIT_ERR_MISALIGNED
+    assert f(0x1000, None, None, 0x2000, 0x3002, 1, 1, 8, 128, None) == dit.DIT_ERR_MISALIGNED
+    g = lib.dit_attn_forward_fp8
+    ok = dict(q=0x1000, k=0x2000, v=0x3000, qs=0x4000, ks=0x5000, vs=0x6000, out=0x7000, lse=None, B=1, H=1,
+              nt=8, ni=8, D=128, dtype=dit.DIT_FP8_E4M3)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["q"], a["k"], a["v"], a["qs"], a["ks"], a["vs"], a["out"], a["lse"], a["B"], a["H"], a["nt"],
+                 a["ni"], a["D"], a["dtype"], None)
+    assert call(v=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(ks=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(nt=0, ni=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(B=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=dit.DIT_BF16) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=dit.DIT_FP8_E4M3 | dit.DIT_K_ROTATED) == dit.DIT_ERR_UNSUPPORTED
+    assert call(q=0x1001) == dit.DIT_ERR_MISALIGNED
+    assert call(vs=0x6002) == dit.DIT_ERR_MISALIGNED
+    assert call(lse=0x8001) == dit.DIT_ERR_MISALIGNED
+
+
 def test_get_status_rejects_null(lib):
     assert lib.dit_attn_get_status(None, None) == dit.DIT_ERR_INVALID_ARG
 
