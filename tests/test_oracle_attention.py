@@ -229,6 +229,38 @@ def test_merge_of_key_slices_equals_full_attention():
     assert np.max(np.abs(o1 - full_o)) < 1e-15 and np.max(np.abs(l1 - full_l)) < 1e-15
 
 
+def test_merge_ignores_empty_key_slices():
+    """A slice with no keys (sum exp = 0, lse = -inf, O = 0/0) changes
+    nothing; the union of empty slices is empty (lse = -inf, O = 0)."""
+    rng = np.random.default_rng(14)
+    N, D = 40, 128
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    full_o, full_l = attention.attention_rows(q, k, v, 1 / math.sqrt(D))
+    nan_o = np.full((N, D), np.nan)
+    ninf = np.full(N, -np.inf)
+    o, l = merge.merge([nan_o, full_o, nan_o], [ninf, full_l, ninf])
+    assert np.array_equal(o, full_o) and np.array_equal(l, full_l)
+    o, l = merge.merge([nan_o, nan_o], [ninf, ninf])
+    assert np.array_equal(o, np.zeros((N, D))) and np.all(np.isneginf(l))
+    # rows that are empty in one part only
+    half = full_l.copy()
+    half[::2] = -np.inf
+    o, l = merge.merge([np.where(np.isneginf(half)[:, None], np.nan, full_o), full_o], [half, full_l])
+    assert np.max(np.abs(o - full_o)) < 1e-15
+    assert np.max(np.abs(l[1::2] - (full_l[1::2] + math.log(2)))) < 1e-13
+    assert np.array_equal(l[::2], full_l[::2])
+
+
+def test_merge_weights_follow_the_softmax_of_the_lses():
+    """Two parts with scalar outputs 0 and 1: O is the logistic function of
+    lse_1 - lse_0, and lse is log(e^a + e^b), both closed forms."""
+    a = np.array([0.0, 3.0, -20.0, 700.0, -700.0])
+    b = np.array([0.0, -1.0, 5.0, 700.5, -699.0])
+    o, l = merge.merge([np.zeros((5, 1)), np.ones((5, 1))], [a, b])
+    assert np.max(np.abs(o[:, 0] - 1.0 / (1.0 + np.exp(a - b)))) < 1e-15
+    assert np.max(np.abs(l - np.logaddexp(a, b))) < 1e-12
+
+
 def test_sampled_rows_equal_the_same_rows_of_the_full_result():
     rng = np.random.default_rng(13)
     B, H, N, D = 2, 3, 70, 128
