@@ -146,6 +146,14 @@ def measured_peaks():
     return FALLBACK_PEAK_BF16, "fallback 1.59 PFLOP/s"
 
 
+def measured_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"])
+    return 6650.0
+
+
 def profile_traffic(kernel_source_sha: str, kernel: str):
     """DRAM bytes per launch of `kernel` on the bench workload from the
     committed ncu summary, or None if none exists for the current source."""
@@ -248,6 +256,48 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
                          "kernel_ms": kern_ms}}
 
 
+def time_merge(args, w, lib, out, lse, stream, dev):
+    """dit_attn_merge of R = 2 bf16 partial results of the workload's shape
+    (a 2-way context-parallel split); memory-bound, reported in GB/s of the
+    algorithmic bytes (R part rows + lses read, one row + lse written)."""
+    import torch
+    import diffusion_transformer_joint_attn_b200 as dit
+    parts = [out, out.clone()]
+    lses = [lse, lse.clone()]
+    merged = torch.empty_like(out)
+    merged_lse = torch.empty_like(lse)
+    R = len(parts)
+    optr = (ctypes.c_void_p * R)(*[p.data_ptr() for p in parts])
+    lptr = (ctypes.c_void_p * R)(*[p.data_ptr() for p in lses])
+    s_ptr = stream.cuda_stream
+
+    def launch():
+        assert lib.dit_attn_merge(ctypes.cast(optr, ctypes.c_void_p), ctypes.cast(lptr, ctypes.c_void_p), R,
+                                  merged.data_ptr(), merged_lse.data_ptr(), w.B, w.H, w.N, w.D, dit.DIT_BF16,
+                                  s_ptr) == 0
+
+    for _ in range(max(3, args.warmup)):
+        launch()
+    steps = max(1, min(args.steps, 50))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        a.record(stream)
+        launch()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    rows = w.B * w.H * w.N
+    nbytes = (R + 1) * rows * (w.D * 2 + 4)
+    peak = measured_hbm()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    # inputs and output (316 MB at 2048^2) exceed the 126 MB L2; no flush between launches
+    return {"R": R, "bytes_per_launch": nbytes, "kernel_ms": ms, "launches": steps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "merge_kernel",
+                         "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
+
+
 # ------------------------------------------------------------------ native arm
 def run_native(args):
     import torch
@@ -318,6 +368,7 @@ def run_native(args):
     value = whole_job_throughput(w.flops, args.steps, world, max_ms)
 
     fp8 = time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, world)
+    merge = time_merge(args, w, lib, out, lse, stream, dev)
 
     # end to end through the public API: pinned host inputs in, O and LSE out
     q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
@@ -382,6 +433,7 @@ def run_native(args):
                     "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": 3 * args.steps,
             "fp8": fp8,
+            "merge": merge,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }

@@ -24,6 +24,8 @@ DIT_FP8_E4M3 = 1
 DIT_OUT_F32 = 0x100
 DIT_K_ROTATED = 0x200
 DIT_V_F16 = 0x400
+DIT_PART_F32 = 0x800
+DIT_MERGE_MAX_PARTS = 16
 
 
 class DitError(RuntimeError):
@@ -173,6 +175,31 @@ def dit_attn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, n_txt:
                                                _stream(stream)), "dit_attn_forward_fp8")
 
 
+def dit_attn_merge(o_parts, lse_parts, out, lse_out=None, dtype: int = DIT_BF16, stream=None) -> None:
+    """out (and lse_out) <- merge of R partial results (lists of [B, H, N, D] outputs and [B, H, N] lses)
+    over disjoint key sets."""
+    import torch
+    R = len(o_parts)
+    _require(1 <= R <= DIT_MERGE_MAX_PARTS and len(lse_parts) == R, "need 1..16 parts with one lse each")
+    B, H, N, D = out.shape
+    part_dtype = torch.float32 if dtype & DIT_PART_F32 else torch.bfloat16
+    for o, l in zip(o_parts, lse_parts):
+        _require(o.is_cuda and o.dtype == part_dtype and o.is_contiguous() and o.shape == out.shape,
+                 "part outputs must be contiguous CUDA tensors of out's shape (fp32 with DIT_PART_F32, else bf16)")
+        _require(l.is_cuda and l.dtype == torch.float32 and l.is_contiguous() and tuple(l.shape) == (B, H, N),
+                 "part lses must be contiguous CUDA fp32 [B, H, N]")
+    out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
+    _require(out.is_cuda and out.dtype == out_dtype and out.is_contiguous(), "out must be contiguous CUDA")
+    if lse_out is not None:
+        _require(lse_out.is_cuda and lse_out.dtype == torch.float32 and lse_out.is_contiguous() and
+                 tuple(lse_out.shape) == (B, H, N), "lse_out must be contiguous CUDA fp32 [B, H, N]")
+    optr = (ctypes.c_void_p * R)(*[o.data_ptr() for o in o_parts])
+    lptr = (ctypes.c_void_p * R)(*[l.data_ptr() for l in lse_parts])
+    _check(load_library().dit_attn_merge(ctypes.cast(optr, ctypes.c_void_p), ctypes.cast(lptr, ctypes.c_void_p), R,
+                                         _ptr(out), _ptr(lse_out), B, H, N, D, dtype, _stream(stream)),
+           "dit_attn_merge")
+
+
 def dit_attn_get_status(stream=None) -> int:
     """Synchronise the stream, return and clear the device status word."""
     st = ctypes.c_int(0)
@@ -204,6 +231,17 @@ def forward(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
     flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0) | (DIT_V_F16 if v_f16 else 0)
     dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt, DIT_BF16 | flags, stream)
+    return out, lse
+
+
+def merge(o_parts, lse_parts, out_f32: bool = False, with_lse: bool = True, stream=None):
+    """Allocate out (and lse) and run dit_attn_merge; returns (out, lse)."""
+    import torch
+    o0 = o_parts[0]
+    out = torch.empty(o0.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=o0.device)
+    lse = torch.empty(o0.shape[:3], dtype=torch.float32, device=o0.device) if with_lse else None
+    flags = (DIT_PART_F32 if o0.dtype == torch.float32 else 0) | (DIT_OUT_F32 if out_f32 else 0)
+    dit_attn_merge(o_parts, lse_parts, out, lse, DIT_BF16 | flags, stream)
     return out, lse
 
 

@@ -20,6 +20,7 @@ SIGNATURES = {
     "dit_attn_forward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_quantize_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
+    "dit_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_get_status": (_I, [ctypes.POINTER(ctypes.c_int), _VP]),
     "dit_attn_status_string": (ctypes.c_char_p, [_I]),
 }

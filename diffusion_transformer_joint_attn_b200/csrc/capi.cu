@@ -145,6 +145,32 @@ int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8
   return dit::launch_attn_fwd_fp8(a, static_cast<cudaStream_t>(stream));
 }
 
+static_assert(DIT_MERGE_MAX_PARTS == dit::kMergeMaxParts, "part limit of the header and the kernel differ");
+
+int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, int R, void* out, float* lse_out,
+                   int B, int H, int N, int D, int dtype, dit_stream_t stream) {
+  if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (R < 1 || R > DIT_MERGE_MAX_PARTS) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if ((dtype & ~(DIT_PART_F32 | DIT_OUT_F32)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+  dit::MergeArgs a;
+  for (int r = 0; r < R; ++r) {
+    if (o_parts[r] == nullptr || lse_parts[r] == nullptr) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(o_parts[r]) || !aligned4(lse_parts[r])) return DIT_ERR_MISALIGNED;
+    a.o[r] = o_parts[r];
+    a.lse[r] = lse_parts[r];
+  }
+  if (!aligned16(out) || (lse_out != nullptr && !aligned4(lse_out))) return DIT_ERR_MISALIGNED;
+  a.R = R;
+  a.out = out;
+  a.lse_out = lse_out;
+  a.rows = static_cast<long long>(B) * H * N;
+  a.in_f32 = (dtype & DIT_PART_F32) != 0;
+  a.out_f32 = (dtype & DIT_OUT_F32) != 0;
+  return dit::launch_merge(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
 int dit_attn_get_status(int* status_host, dit_stream_t stream) {
   if (status_host == nullptr) return DIT_ERR_INVALID_ARG;
   int* word = dit::device_status_word();

@@ -78,6 +78,18 @@ struct AttnFwdFp8Args {
 };
 int launch_attn_fwd_fp8(const AttnFwdFp8Args& a, cudaStream_t s);
 
+constexpr int kMergeMaxParts = 16;
+struct MergeArgs {
+  const void* o[kMergeMaxParts];      // part outputs [rows][128], bf16 or fp32
+  const float* lse[kMergeMaxParts];   // part log-sum-exps [rows]
+  int R;
+  void* out;
+  float* lse_out;                     // may be null
+  long long rows;
+  bool in_f32, out_f32;
+};
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
+
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s);

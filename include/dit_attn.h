@@ -57,6 +57,8 @@ typedef enum { DIT_BF16 = 0, DIT_FP8_E4M3 = 1 } dit_dtype_t;
 #define DIT_OUT_F32 0x100   /* write `out` as fp32 instead of bf16 */
 #define DIT_K_ROTATED 0x200 /* k already carries the rotary embedding (dit_rope_apply); rotate q only */
 #define DIT_V_F16 0x400     /* v is given as fp16 (dit_attn_prepare_kv) instead of bf16 */
+#define DIT_PART_F32 0x800  /* dit_attn_merge: the part outputs are fp32 instead of bf16 */
+#define DIT_MERGE_MAX_PARTS 16
 
 /*
  * dit_rope_table_build — cos/sin table of the three-axis rotary embedding.
@@ -198,6 +200,34 @@ int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float
 int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* q_scale,
                          const float* k_scale, const float* v_scale, void* out, float* lse, int B, int H,
                          int N_txt, int N_img, int D, int dtype, dit_stream_t stream);
+
+/*
+ * dit_attn_merge — combine R partial results of the same queries over
+ * disjoint key sets into the result over their union (context parallelism:
+ * wavespeed.ai "Beschleunigung der FLUX.1-dev Bildgenerierung", section on
+ * context parallelism and First Block Cache):
+ *     lse = ln sum_r exp(lse_r),   out = sum_r exp(lse_r - lse) O_r.
+ *
+ *   o_parts   HOST array of R device pointers, each [B][H][N][D] bf16 (fp32
+ *             with DIT_PART_F32): the normalised partial outputs, as
+ *             dit_attn_forward writes them.
+ *   lse_parts HOST array of R device pointers, each [B][H][N] fp32.  A part
+ *             with lse = -inf has no keys: its weight is 0 and the values of
+ *             its output row are not used (they may be NaN; the memory must
+ *             still be readable).
+ *   R         1 .. DIT_MERGE_MAX_PARTS.
+ *   out       device [B][H][N][D], bf16 (fp32 with DIT_OUT_F32).  Rows whose
+ *             parts are all empty get 0.  May be the same buffer as one of
+ *             the parts (same dtype): each element is read before written.
+ *   lse_out   device fp32 [B][H][N] or NULL; may be one of lse_parts.
+ *   dtype     DIT_BF16, optionally | DIT_PART_F32 | DIT_OUT_F32.
+ * The parts may be in another GPU's memory if that memory is accessible from
+ * the current device (peer access enabled or an imported IPC mapping): the
+ * kernel reads them with ordinary loads.  Weights use expf / logf in fp32.
+ * Alignment: parts and out 16 bytes, lse arrays 4 bytes.  D must be 128.
+ */
+int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, int R, void* out, float* lse_out,
+                   int B, int H, int N, int D, int dtype, dit_stream_t stream);
 
 /*
  * dit_attn_get_status — synchronise `stream`, copy the device status word to

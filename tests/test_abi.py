@@ -129,6 +129,28 @@ def test_fp8_argument_errors(lib):
     assert call(lse=0x8001) == dit.DIT_ERR_MISALIGNED
 
 
+def test_merge_argument_errors(lib):
+    f = lib.dit_attn_merge
+
+    def call(R=2, o=(0x1000, 0x2000), l=(0x3000, 0x4000), out=0x5000, lse=None, B=1, H=1, N=8, D=128, dtype=0):
+        oa = (ctypes.c_void_p * max(len(o), 1))(*o)
+        la = (ctypes.c_void_p * max(len(l), 1))(*l)
+        return f(ctypes.cast(oa, ctypes.c_void_p), ctypes.cast(la, ctypes.c_void_p), R, out, lse, B, H, N, D, dtype,
+                 None)
+    assert f(None, None, 1, 0x5000, None, 1, 1, 8, 128, 0, None) == dit.DIT_ERR_INVALID_ARG
+    assert call(R=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(R=17, o=(0x1000,) * 17, l=(0x3000,) * 17) == dit.DIT_ERR_INVALID_ARG
+    assert call(o=(0x1000, None)) == dit.DIT_ERR_INVALID_ARG
+    assert call(out=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(N=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=dit.DIT_FP8_E4M3) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=dit.DIT_K_ROTATED) == dit.DIT_ERR_UNSUPPORTED
+    assert call(o=(0x1000, 0x2008)) == dit.DIT_ERR_MISALIGNED
+    assert call(l=(0x3000, 0x4002)) == dit.DIT_ERR_MISALIGNED
+    assert call(lse=0x6001) == dit.DIT_ERR_MISALIGNED
+
+
 def test_get_status_rejects_null(lib):
     assert lib.dit_attn_get_status(None, None) == dit.DIT_ERR_INVALID_ARG
 
