@@ -294,7 +294,9 @@ def time_merge(args, w, lib, out, lse, stream, dev):
     # inputs and output (316 MB at 2048^2) exceed the 126 MB L2; no flush between launches
     return {"R": R, "bytes_per_launch": nbytes, "kernel_ms": ms, "launches": steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "merge_kernel",
+                         "frac": achieved / peak, "kernel": "merge_kernel",
+                         "traffic": profile_traffic(kernel_source_sha(), "merge_kernel") if w.name == WORKLOAD
+                         else None,
                          "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
 
 

@@ -31,7 +31,11 @@ DIT_MERGE_MAX_PARTS = 16
 class DitError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__("%s failed: %s (%d)" % (what, dit_attn_status_string(status), status))
+        msg = "%s failed: %s (%d)" % (what, dit_attn_status_string(status), status)
+        if status == DIT_ERR_CUDA:
+            lib = load_library()
+            msg += ": %s (%d)" % (lib.dit_attn_last_cuda_error_string().decode(), lib.dit_attn_last_cuda_error())
+        super().__init__(msg)
 
 
 def _check(status: int, what: str) -> None:

@@ -54,12 +54,13 @@ __device__ __forceinline__ float max64(const float* f) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// P for 64 consecutive logits of the row: 2^(s c - m c) rounded to fp16, packed
-// in pairs into pk[32]; adds the rounded values to sum[4].
-__device__ __forceinline__ void exp_half(const float* f, float c, float neg, uint32_t* pk, float* sum) {
+// P for 2 kPairs consecutive logits of the row: 2^(s c - m c) rounded to
+// fp16, packed in pairs into pk[kPairs]; adds the rounded values to sum[4].
+template <int kPairs>
+__device__ __forceinline__ void exp_pairs(const float* f, float c, float neg, uint32_t* pk, float* sum) {
   const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < kPairs; ++i) {
     const float2 x = __ffma2_rn(make_float2(f[2 * i], f[2 * i + 1]), c2, n2);
     float e0, e1;
     if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
@@ -73,6 +74,9 @@ __device__ __forceinline__ void exp_half(const float* f, float c, float neg, uin
     // dominated by one key returns that key's V row exactly
     sum[i & 3] = add_f16x2_to_f32(sum[i & 3], pk[i]);
   }
+}
+__device__ __forceinline__ void exp_half(const float* f, float c, float neg, uint32_t* pk, float* sum) {
+  exp_pairs<32>(f, c, neg, pk, sum);
 }
 
 // Barriers, outputs and (FP8 only) block scales of one CTA's softmax warps.
@@ -181,7 +185,7 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
   if (ok && warp_wait(&io.o_final[t], 0, wc)) {
     tc_fence_after();
     const bool valid = n < io.N;
-    const float inv_l = 1.0f / l;
+    const float inv_l = __frcp_rn(l);        // reciprocal without the division slow-path call
     const size_t row_off = (static_cast<size_t>(pr.bh) * io.N + n) * kHeadDim;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -213,6 +217,7 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
     }
   }
 }
+
 
 }  // namespace attn
 }  // namespace dit

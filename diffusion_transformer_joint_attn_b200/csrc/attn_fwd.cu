@@ -64,8 +64,9 @@ struct __align__(1024) Smem {
   uint8_t v[kStages][kVHalfBytes];
   uint64_t q_full;
   uint64_t q_ready;                                   // even CTA: one arrive per CTA
-  uint64_t k_full[kStages], k_ready[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_ready[kStages], v_empty[kStages];
+  uint64_t k_full[kStages], k_ready[kStages];
+  uint64_t v_full[kStages], v_ready[kStages];
+  uint64_t kv_empty[kStages];                          // stage s free again: P V of its tile has completed
   uint64_t s_full[2], p_ready[2], o_final[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -183,7 +184,7 @@ __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const C
     const int s = j % kStages;
     const uint32_t ph = (j / kStages) & 1;
     const int key0 = j * kTile;
-    if (!mbar_wait(&sm.k_empty[s], ph ^ 1, wc)) break;
+    if (!mbar_wait(&sm.kv_empty[s], ph ^ 1, wc)) break;
     if (kPrepared) {
       if (leader) mbar_arrive_expect_tx(&sm.k_full[s], 2 * kKHalfBytes);
       const uint32_t bar = cl(&sm.k_full[s], 0);
@@ -194,10 +195,6 @@ __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const C
       for (int b = 0; b < 2; ++b)
         tma_load_3d(sm.k[s] + b * kKBoxBytes, tm_k, &sm.k_full[s], b * 64, key0 + 64 * static_cast<int>(pr.rank),
                     pr.bh);
-    }
-    if (!mbar_wait(&sm.v_empty[s], ph ^ 1, wc)) {
-      issued = 2 * j + 1;
-      break;
     }
     if (kPrepared) {
       if (leader) mbar_arrive_expect_tx(&sm.v_full[s], 2 * kVHalfBytes);
@@ -281,8 +278,8 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
       }
     }
     if (!ok) break;
-    if (j < p.n_kv) commit_both(&sm.k_empty[s]);
-    if (j > 0) commit_both(&sm.v_empty[sp]);
+    // one release per stage: the commit tracks Q K_{j-1}^T and P V_{j-1}
+    if (j > 0) commit_both(&sm.kv_empty[sp]);
   }
   // every MMA issued above has completed once this arrives
   tc_commit_pair(cl(&sm.mma_drain, 0));
@@ -351,10 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_ready[s], 2 * kProWarps);
-      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_ready[s], 2 * kProWarps);
-      mbar_init(&sm.v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);

@@ -46,9 +46,10 @@ struct __align__(1024) Smem {
   uint8_t v8[kStages][kV8HalfBytes];
   uint8_t v[kStages][kVHalfBytes];
   uint64_t q_full;                                   // even CTA: both CTAs' Q codes
-  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t k_full[kStages];
+  uint64_t kv_empty[kStages];                        // stage s free again: P V of its tile has completed
   uint64_t v8_full[kStages], v8_empty[kStages];      // local staging ring
-  uint64_t v_ready[kStages], v_empty[kStages];
+  uint64_t v_ready[kStages];
   uint64_t s_full[2], p_ready[2], o_final[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -84,7 +85,7 @@ __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const C
     const int s = j % kStages;
     const uint32_t ph = (j / kStages) & 1;
     const int key0 = j * kTile;
-    if (!mbar_wait(&sm.k_empty[s], ph ^ 1, wc)) break;
+    if (!mbar_wait(&sm.kv_empty[s], ph ^ 1, wc)) break;
     if (leader) mbar_arrive_expect_tx(&sm.k_full[s], 2 * kK8HalfBytes);
     tma_load_3d_pair(sm.k[s], tm_k, cl(&sm.k_full[s], 0), 0, key0 + 64 * static_cast<int>(pr.rank), pr.bh);
     if (!mbar_wait(&sm.v8_empty[s], ph ^ 1, wc)) {
@@ -154,8 +155,8 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
       }
     }
     if (!ok) break;
-    if (j < p.n_kv) commit_both(&sm.k_empty[s]);
-    if (j > 0) commit_both(&sm.v_empty[sp]);
+    // one release per stage: the commit tracks Q K_{j-1}^T and P V_{j-1}
+    if (j > 0) commit_both(&sm.kv_empty[sp]);
   }
   tc_commit_pair(cl(&sm.mma_drain, 0));
   mbar_wait_drain(&sm.mma_drain, 0, wc);
@@ -178,7 +179,7 @@ __device__ __forceinline__ void dequant_v_role(Smem& sm, const Params& p, const 
     const int s = j % kStages;
     const uint32_t ph = (j / kStages) & 1;
     if (!warp_wait(&sm.v8_full[s], ph, wc)) break;
-    if (!warp_wait(&sm.v_empty[s], ph ^ 1, wc)) break;
+    if (!warp_wait(&sm.kv_empty[s], ph ^ 1, wc)) break;
     const int blk0 = 2 * j;
     const float vs0 = __ldg(vscale + blk0);
     const float vs1 = blk0 + 1 < p.n_blocks ? __ldg(vscale + blk0 + 1) : vs0;
@@ -222,11 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
       mbar_init(&sm.v8_full[s], 1);
       mbar_init(&sm.v8_empty[s], kCvtWarps);
       mbar_init(&sm.v_ready[s], 2 * kCvtWarps);
-      mbar_init(&sm.v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);

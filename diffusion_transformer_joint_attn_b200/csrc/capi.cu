@@ -49,6 +49,21 @@ namespace {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// CUDA runtime error behind the last DIT_ERR_CUDA of this host thread.
+thread_local int t_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DIT_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return DIT_ERR_CUDA;
+}
+// For launchers that return a dit_status_t: on DIT_ERR_CUDA take (and clear)
+// the runtime's last error.
+int launcher_status(int rc) {
+  if (rc == DIT_ERR_CUDA) t_last_cuda_error = static_cast<int>(cudaGetLastError());
+  return rc;
+}
+
 }  // namespace
 
 extern "C" {
@@ -64,7 +79,7 @@ int dit_rope_table_build(const int32_t* pos, int N, int D, const int32_t* axes, 
   if (static_cast<long long>(N) * (D / 2) > (1LL << 40)) return DIT_ERR_INVALID_ARG;
   if (!aligned4(pos) || !aligned16(rope_cos) || !aligned16(rope_sin)) return DIT_ERR_MISALIGNED;
   dit::RopeTableArgs a{pos, N, D, {axes[0], axes[1], axes[2]}, theta, rope_cos, rope_sin};
-  return dit::launch_rope_table(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  return cuda_status(dit::launch_rope_table(a, static_cast<cudaStream_t>(stream)));
 }
 
 int dit_rope_apply(const void* x, const float* rope_cos, const float* rope_sin, void* x_rot, int B, int H, int N,
@@ -75,7 +90,7 @@ int dit_rope_apply(const void* x, const float* rope_cos, const float* rope_sin, 
   if (D != 128) return DIT_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(x_rot) || !aligned16(rope_cos) || !aligned16(rope_sin)) return DIT_ERR_MISALIGNED;
   dit::RopeApplyArgs a{x, rope_cos, rope_sin, x_rot, B, H, N, D};
-  return dit::launch_rope_apply(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  return cuda_status(dit::launch_rope_apply(a, static_cast<cudaStream_t>(stream)));
 }
 
 int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, const float* rope_sin, void* k_rot,
@@ -90,7 +105,7 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
       !aligned16(rope_sin))
     return DIT_ERR_MISALIGNED;
   dit::PrepareKVArgs a{k, v, rope_cos, rope_sin, k_rot, v_f16, B, H, N, D};
-  return dit::launch_prepare_kv(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  return cuda_status(dit::launch_prepare_kv(a, static_cast<cudaStream_t>(stream)));
 }
 
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
@@ -110,7 +125,7 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
     return DIT_ERR_MISALIGNED;
   dit::AttnFwdArgs a{q,   k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N), (dtype & DIT_OUT_F32) != 0,
                      (dtype & DIT_K_ROTATED) != 0, (dtype & DIT_V_F16) != 0};
-  return dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream));
+  return launcher_status(dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
 }
 
 int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float* rope_sin, uint8_t* x_fp8,
@@ -123,7 +138,7 @@ int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float
   if (!aligned16(x_bf16) || !aligned16(x_fp8) || !aligned4(scale)) return DIT_ERR_MISALIGNED;
   if (rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) return DIT_ERR_MISALIGNED;
   dit::QuantFp8Args a{x_bf16, rope_cos, rope_sin, x_fp8, scale, B, H, N};
-  return dit::launch_quantize_fp8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  return cuda_status(dit::launch_quantize_fp8(a, static_cast<cudaStream_t>(stream)));
 }
 
 int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* q_scale,
@@ -142,7 +157,7 @@ int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8
     return DIT_ERR_MISALIGNED;
   dit::AttnFwdFp8Args a{q8, k8, v8, q_scale, k_scale, v_scale, out, lse, B, H, static_cast<int>(N),
                         (dtype & DIT_OUT_F32) != 0};
-  return dit::launch_attn_fwd_fp8(a, static_cast<cudaStream_t>(stream));
+  return launcher_status(dit::launch_attn_fwd_fp8(a, static_cast<cudaStream_t>(stream)));
 }
 
 static_assert(DIT_MERGE_MAX_PARTS == dit::kMergeMaxParts, "part limit of the header and the kernel differ");
@@ -168,7 +183,7 @@ int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, in
   a.rows = static_cast<long long>(B) * H * N;
   a.in_f32 = (dtype & DIT_PART_F32) != 0;
   a.out_f32 = (dtype & DIT_OUT_F32) != 0;
-  return dit::launch_merge(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  return cuda_status(dit::launch_merge(a, static_cast<cudaStream_t>(stream)));
 }
 
 int dit_attn_get_status(int* status_host, dit_stream_t stream) {
@@ -177,11 +192,18 @@ int dit_attn_get_status(int* status_host, dit_stream_t stream) {
   if (word == nullptr) return DIT_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int value = 0;
-  if (cudaMemcpyAsync(&value, word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return DIT_ERR_CUDA;
-  if (cudaMemsetAsync(word, 0, sizeof(int), s) != cudaSuccess) return DIT_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return DIT_ERR_CUDA;
+  int rc = cuda_status(cudaMemcpyAsync(&value, word, sizeof(int), cudaMemcpyDeviceToHost, s));
+  if (rc == DIT_OK) rc = cuda_status(cudaMemsetAsync(word, 0, sizeof(int), s));
+  if (rc == DIT_OK) rc = cuda_status(cudaStreamSynchronize(s));
+  if (rc != DIT_OK) return rc;
   *status_host = value;
   return DIT_OK;
+}
+
+int dit_attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char* dit_attn_last_cuda_error_string(void) {
+  return cudaGetErrorString(static_cast<cudaError_t>(t_last_cuda_error));
 }
 
 const char* dit_attn_status_string(int status) {

@@ -237,6 +237,17 @@ int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, in
  */
 int dit_attn_get_status(int* status_host, dit_stream_t stream);
 
+/*
+ * dit_attn_last_cuda_error — the CUDA runtime error code (a cudaError_t)
+ * behind the most recent DIT_ERR_CUDA returned to this host thread, or 0 if
+ * there was none or the failing call was a driver call that leaves no runtime
+ * error (the tensor-map encoding).  dit_attn_last_cuda_error_string gives the
+ * runtime's description of that code.  Neither makes a CUDA call that can
+ * fail; both may be called without a GPU.
+ */
+int dit_attn_last_cuda_error(void);
+const char* dit_attn_last_cuda_error_string(void);
+
 /* Static English description of a dit_status_t value. */
 const char* dit_attn_status_string(int status);
 

@@ -41,6 +41,9 @@ def test_status_strings(lib):
     assert dit.dit_attn_status_string(0) == "ok"
     assert "timed out" in dit.dit_attn_status_string(-5)
     assert dit.dit_attn_status_string(12345) == "unknown status"
+    # no CUDA call has failed in this process: no recorded runtime error
+    assert lib.dit_attn_last_cuda_error() == 0
+    assert lib.dit_attn_last_cuda_error_string() == b"no error"
 
 
 def _fwd(lib, q=0x10000, k=0x20000, v=0x30000, cos=None, sin=None, out=0x40000, lse=None, B=1, H=1, nt=8, ni=8, D=128,
