@@ -23,6 +23,12 @@ for intermediate values, with exact arithmetic in between:
   bf16 (ties to even): the operand precision of a bf16 tensor-core product.
 Everything else stays fp64.
 
+With `kv_mask` the sum runs over the keys of the allowed (query block, key
+tile) pairs only: the block-sparse form that skips whole tiles (a generic
+stand-in for the sparse attention the pages name as prior art: scopeai.cc,
+section on each optimisation's effect; bpdata.com, section on the reference
+kernels).
+
 Test infrastructure only (see oracle/__init__.py).
 """
 from __future__ import annotations
@@ -40,14 +46,28 @@ def to_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def attention_rows(q_rows, k, v, scale):
-    """softmax(q_rows k^T * scale) v for one (b, h): returns O [R, D], LSE [R]."""
+def attention_rows(q_rows, k, v, scale, allowed=None):
+    """softmax(q_rows k^T * scale) v for one (b, h): returns O [R, D], LSE [R].
+
+    allowed: optional bool [R, N], the keys each row attends to; the others
+    are left out of the softmax (their logits taken as -inf).  A row with no
+    key has an empty sum: O = 0 and LSE = -inf.
+    """
     s = (q_rows @ k.T) * scale
+    if allowed is not None:
+        s = np.where(allowed, s, -np.inf)
+        empty = ~allowed.any(axis=1)
+        s[empty] = 0.0                       # placeholder logits, result replaced below
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
+    if allowed is not None:
+        e = np.where(allowed | empty[:, None], e, 0.0)
     l = e.sum(axis=1, keepdims=True)
     out = (e @ v) / l
     lse = m[:, 0] + np.log(l[:, 0])
+    if allowed is not None:
+        out[empty] = 0.0
+        lse[empty] = -np.inf
     return out, lse
 
 
@@ -69,11 +89,16 @@ def _round(x, how):
 
 
 def joint_attention(q, k, v, pos=None, rows=None, axes=rope.DEFAULT_AXES,
-                    theta: float = rope.DEFAULT_THETA, scale=None, round_rotated=None, table_fp32=False):
+                    theta: float = rope.DEFAULT_THETA, scale=None, round_rotated=None, table_fp32=False,
+                    kv_mask=None, q_block: int = 512, kv_block: int = 128):
     """Oracle output for tensors q, k, v [B, H, N, D].
 
     pos:  int [N, 3] token positions (t, h, w) or None for no rotary embedding.
     rows: int [R, 3] (b, h, n) query rows to evaluate, or None for all rows.
+    kv_mask: optional [B, H, ceil(N / q_block), ceil(N / kv_block)] array:
+          query n of (b, h) attends to key m only where
+          kv_mask[b, h, n // q_block, m // kv_block] is nonzero (block-sparse
+          attention; the selection rule is the caller's).
     Returns (O [R, D], LSE [R]) in fp64, in the order of `rows` (row-major
     (b, h, n) order when rows is None).
     """
@@ -101,7 +126,11 @@ def joint_attention(q, k, v, pos=None, rows=None, axes=rope.DEFAULT_AXES,
             qq = rope.rotate_with_table(qq, cs[0][rows[idx, 2]], cs[1][rows[idx, 2]])
         kk = _round(kk, round_rotated)
         qq = _round(qq, round_rotated)
-        o, l = attention_rows(qq, kk, vv, scale)
+        allowed = None
+        if kv_mask is not None:
+            blocks = np.asarray(kv_mask)[bb, hh] != 0                       # [n_qblk, n_kvblk]
+            allowed = blocks[rows[idx, 2] // q_block][:, np.arange(N) // kv_block]
+        o, l = attention_rows(qq, kk, vv, scale, allowed)
         out[idx] = o
         lse[idx] = l
     return out, lse

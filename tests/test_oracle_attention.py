@@ -261,6 +261,64 @@ def test_merge_weights_follow_the_softmax_of_the_lses():
     assert np.max(np.abs(l - np.logaddexp(a, b))) < 1e-12
 
 
+# --------------------------------------------------------------- block-sparse pins
+
+def _sparse_case(seed=21, B=1, H=2, N=700):
+    rng = np.random.default_rng(seed)
+    q, k, v = (rng.standard_normal((B, H, N, 128)) for _ in range(3))
+    pos = rng.integers(0, 40, size=(N, 3))
+    nq, nk = -(-N // 512), -(-N // 128)
+    return rng, q, k, v, pos, nq, nk
+
+
+def test_all_ones_mask_is_dense_attention():
+    rng, q, k, v, pos, nq, nk = _sparse_case()
+    O, L = attention.joint_attention(q, k, v, pos=pos)
+    Os, Ls = attention.joint_attention(q, k, v, pos=pos, kv_mask=np.ones((1, 2, nq, nk), np.uint8))
+    assert np.array_equal(O, Os) and np.array_equal(L, Ls)
+
+
+def test_single_tile_mask_is_attention_over_that_key_slice():
+    rng, q, k, v, pos, nq, nk = _sparse_case()
+    mask = np.zeros((1, 2, nq, nk), np.uint8)
+    mask[0, 1, 0, 5] = 1                 # rows 0..511 of head 1 see keys 640..699 (the ragged last tile)
+    mask[0, 1, 1, 2] = 1                 # rows 512..699 of head 1 see keys 256..383
+    rows = np.array([[0, 1, 3], [0, 1, 511], [0, 1, 512], [0, 1, 699]])
+    O, L = attention.joint_attention(q, k, v, pos=pos, rows=rows, kv_mask=mask)
+    ang = rope.angles(pos)
+    qr, kr = rope.rotate(q[0, 1], ang), rope.rotate(k[0, 1], ang)
+    for i, (lo, hi) in enumerate([(640, 700), (640, 700), (256, 384), (256, 384)]):
+        o, l = attention.attention_rows(qr[rows[i, 2]][None], kr[lo:hi], v[0, 1, lo:hi], 1 / math.sqrt(128))
+        assert np.max(np.abs(O[i] - o[0])) < 1e-13 and abs(L[i] - l[0]) < 1e-12
+
+
+def test_rows_without_keys_are_zero_with_minus_infinite_lse():
+    rng, q, k, v, pos, nq, nk = _sparse_case()
+    mask = np.ones((1, 2, nq, nk), np.uint8)
+    mask[0, 0, 1, :] = 0
+    O, L = attention.joint_attention(q, k, v, pos=pos, kv_mask=mask)
+    O = O.reshape(1, 2, 700, 128)
+    L = L.reshape(1, 2, 700)
+    assert np.all(O[0, 0, 512:] == 0) and np.all(np.isneginf(L[0, 0, 512:]))
+    assert np.all(np.isfinite(L[0, 0, :512])) and np.all(np.isfinite(L[0, 1]))
+
+
+def test_complementary_masks_merge_to_dense_attention():
+    """Splitting the key tiles of every row between two masks and merging the
+    two block-sparse results gives the dense result: ties the block-sparse
+    definition to the merge of partial results."""
+    rng, q, k, v, pos, nq, nk = _sparse_case()
+    m1 = rng.integers(0, 2, size=(1, 2, nq, nk)).astype(np.uint8)
+    m1[0, 0, 0, :] = 0                   # one block entirely in the other part
+    m2 = 1 - m1
+    O, L = attention.joint_attention(q, k, v, pos=pos)
+    O1, L1 = attention.joint_attention(q, k, v, pos=pos, kv_mask=m1)
+    O2, L2 = attention.joint_attention(q, k, v, pos=pos, kv_mask=m2)
+    Om, Lm = merge.merge([O1, O2], [L1, L2])
+    assert np.max(np.abs(Om - O)) < 1e-13
+    assert np.max(np.abs(Lm - L)) < 1e-12
+
+
 def test_sampled_rows_equal_the_same_rows_of_the_full_result():
     rng = np.random.default_rng(13)
     B, H, N, D = 2, 3, 70, 128
