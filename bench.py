@@ -256,6 +256,46 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
                          "kernel_ms": kern_ms}}
 
 
+def time_sparse(args, w, lib, q, k_rot, v_f16, cos, sin, out, lse, stream, dev, dense_ms, density=0.5):
+    """dit_attn_forward_sparse on the same prepared operands with a seeded
+    random block mask selecting `density` of the (512-row query block,
+    128-key tile) pairs.  Throughput counts the selected work only (4 x
+    rows x keys x D per selected pair, ragged edges exact)."""
+    import torch
+    nq, nk = (w.N + 511) // 512, (w.N + 127) // 128
+    rng = np.random.default_rng(0)
+    mask = (rng.random((w.B, w.H, nq, nk)) < density).astype(np.uint8)
+    rows = np.minimum(512, w.N - 512 * np.arange(nq))
+    keys = np.minimum(128, w.N - 128 * np.arange(nk))
+    flops = 4.0 * w.D * float((mask * rows[None, None, :, None] * keys[None, None, None, :]).sum())
+    md = torch.from_numpy(mask).to(dev)
+    flags = 0x200 | 0x400          # DIT_K_ROTATED | DIT_V_F16
+    s_ptr = stream.cuda_stream
+
+    def launch():
+        assert lib.dit_attn_forward_sparse(q.data_ptr(), k_rot.data_ptr(), v_f16.data_ptr(), cos.data_ptr(),
+                                           sin.data_ptr(), md.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B, w.H,
+                                           w.n_txt, w.n_img, w.D, flags, s_ptr) == 0
+
+    for _ in range(max(3, args.warmup)):
+        launch()
+    steps = max(1, min(args.steps, 30))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        a.record(stream)
+        launch()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    peak, src = measured_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"density": float(mask.mean()), "kernel_ms": ms, "time_vs_dense": ms / dense_ms, "launches": steps,
+            "selected_tflop": flops / 1e12,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                         "traffic": None, "kernel": "attn_fwd_bf16_kernel (block-sparse)", "peak_source": src}}
+
+
 def time_merge(args, w, lib, out, lse, stream, dev):
     """dit_attn_merge of R = 2 bf16 partial results of the workload's shape
     (a 2-way context-parallel split); memory-bound, reported in GB/s of the
@@ -371,6 +411,7 @@ def run_native(args):
 
     fp8 = time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, world)
     merge = time_merge(args, w, lib, out, lse, stream, dev)
+    sparse = time_sparse(args, w, lib, q, k_rot, v_f16, cos, sin, out, lse, stream, dev, kern_ms)
 
     # end to end through the public API: pinned host inputs in, O and LSE out
     q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
@@ -436,6 +477,7 @@ def run_native(args):
             "gpu_launches": 3 * args.steps,
             "fp8": fp8,
             "merge": merge,
+            "sparse": sparse,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }

@@ -26,6 +26,7 @@ DIT_K_ROTATED = 0x200
 DIT_V_F16 = 0x400
 DIT_PART_F32 = 0x800
 DIT_MERGE_MAX_PARTS = 16
+DIT_SPARSE_MAX_KV_TILES = 4096
 
 
 class DitError(RuntimeError):
@@ -105,6 +106,14 @@ def dit_attn_prepare_kv(k, v, rope_cos, rope_sin, k_rot, v_f16, stream=None) -> 
 def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: int, dtype: int = DIT_BF16,
                      stream=None) -> None:
     """out (and lse, if not None) <- joint attention of bf16 q, k, v [B, H, N, D] on the GPU."""
+    B, H, N, D = q.shape
+    _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dtype)
+    _check(load_library().dit_attn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(out),
+                                           _ptr(lse), B, H, n_txt, n_img, D, dtype, _stream(stream)),
+           "dit_attn_forward")
+
+
+def _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dtype):
     import torch
     _require(q.dim() == 4 and q.shape == k.shape == v.shape, "q, k, v must share one [B, H, N, D] shape")
     B, H, N, D = q.shape
@@ -123,9 +132,21 @@ def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: i
         for t in (rope_cos, rope_sin):
             _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
                      tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
-    _check(load_library().dit_attn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(out),
-                                           _ptr(lse), B, H, n_txt, n_img, D, dtype, _stream(stream)),
-           "dit_attn_forward")
+
+
+def dit_attn_forward_sparse(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, n_txt: int, n_img: int,
+                            dtype: int = DIT_BF16, stream=None) -> None:
+    """dit_attn_forward restricted to the key tiles of kv_mask (CUDA uint8
+    [B, H, ceil(N/512), ceil(N/128)], nonzero = attend)."""
+    import torch
+    B, H, N, D = q.shape
+    _require(kv_mask is not None and kv_mask.is_cuda and kv_mask.dtype == torch.uint8 and kv_mask.is_contiguous()
+             and tuple(kv_mask.shape) == (B, H, (N + 511) // 512, (N + 127) // 128),
+             "kv_mask must be a contiguous CUDA uint8 [B, H, ceil(N/512), ceil(N/128)] tensor")
+    _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dtype)
+    _check(load_library().dit_attn_forward_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
+                                                  _ptr(kv_mask), _ptr(out), _ptr(lse), B, H, n_txt, n_img, D, dtype,
+                                                  _stream(stream)), "dit_attn_forward_sparse")
 
 
 def dit_attn_quantize_fp8(x, rope_cos, rope_sin, x_fp8, scale, stream=None) -> None:
@@ -246,6 +267,19 @@ def merge(o_parts, lse_parts, out_f32: bool = False, with_lse: bool = True, stre
     lse = torch.empty(o0.shape[:3], dtype=torch.float32, device=o0.device) if with_lse else None
     flags = (DIT_PART_F32 if o0.dtype == torch.float32 else 0) | (DIT_OUT_F32 if out_f32 else 0)
     dit_attn_merge(o_parts, lse_parts, out, lse, DIT_BF16 | flags, stream)
+    return out, lse
+
+
+def forward_sparse(q, k, v, kv_mask, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool = False,
+                   with_lse: bool = True, k_rotated: bool = False, v_f16: bool = False, stream=None):
+    """Allocate out (and lse) and run dit_attn_forward_sparse; returns (out, lse)."""
+    import torch
+    B, H, N, D = q.shape
+    out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
+    flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0) | (DIT_V_F16 if v_f16 else 0)
+    dit_attn_forward_sparse(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, n_txt, N - n_txt, DIT_BF16 | flags,
+                            stream)
     return out, lse
 
 

@@ -18,6 +18,7 @@ SIGNATURES = {
     "dit_rope_apply": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_prepare_kv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
+    "dit_attn_forward_sparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_quantize_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _VP]),

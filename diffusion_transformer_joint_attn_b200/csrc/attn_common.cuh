@@ -93,6 +93,8 @@ struct SoftmaxIo {
   const float* q_scale;    // this (b, h)'s per-64-token scales, or nullptr (unscaled logits)
   const float* k_scale;
   int n_blocks;            // ceil(N / 64)
+  const uint16_t* kv_list; // key tiles visited, in order (block-sparse instances only)
+  int n_act;               // number of key tiles visited
 };
 
 // Online softmax of this CTA's tile of slot t, then the epilogue (warps 4-11).
@@ -104,7 +106,7 @@ struct SoftmaxIo {
 // raised only when a tile's maximum exceeds it by more than 8 (log2 units),
 // so P stays in [0, 256]; the raise rescales O in tensor memory and is
 // warp-uniform because tcgen05 loads / stores are warp-collective.
-template <bool kScaled>
+template <bool kScaled, bool kSparse = false>
 __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem, const Pair& pr, int warp, int lane,
                                              const WaitCtx& wc) {
   const int t = (warp - 4) >> 2;
@@ -122,7 +124,8 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
   if (kScaled && n < io.N) qs = __ldg(io.q_scale + n / 64);
   float m_used = 0.f, l = 0.f;
   bool ok = true;
-  for (int j = 0; j < io.n_kv; ++j) {
+  for (int i = 0; i < io.n_act; ++i) {
+    const int j = kSparse ? static_cast<int>(io.kv_list[i]) : i;   // key tile
     float sc0 = 1.0f, sc1 = 1.0f;
     if (kScaled) {
       const float ks0 = __ldg(io.k_scale + 2 * j);
@@ -130,7 +133,7 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
       sc0 = qs * ks0;
       sc1 = qs * ks1;
     }
-    if (!(ok = warp_wait(&io.s_full[t], j & 1, wc))) break;
+    if (!(ok = warp_wait(&io.s_full[t], i & 1, wc))) break;
     tc_fence_after();
     uint32_t s[128];
 #pragma unroll
@@ -138,15 +141,15 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
 #pragma unroll
     for (int q = 0; q < 4; ++q) tmem_ld_wait(s + q * 32);
     float* f = reinterpret_cast<float*>(s);
-    if (j == io.n_kv - 1 && last_valid < kTile) {
+    if (j == io.n_kv - 1 && last_valid < kTile) {     // keys past N in the last tile
 #pragma unroll
-      for (int i = 0; i < 128; ++i)
-        if (i >= last_valid) f[i] = -INFINITY;
+      for (int e = 0; e < 128; ++e)
+        if (e >= last_valid) f[e] = -INFINITY;
     }
     const float mx = kScaled ? fmaxf(max64(f) * sc0, max64(f + 64) * sc1) : fmaxf(max64(f), max64(f + 64));
     float alpha = 1.0f;
     bool rescale = false;
-    if (j == 0) {
+    if (i == 0) {
       m_used = mx;
     } else if (__any_sync(0xffffffffu, mx > m_used + rescale_gap)) {
       const float m_new = fmaxf(m_used, mx);
@@ -181,17 +184,23 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
     __syncwarp();
     if (lane == 0) mbar_arrive_remote(p_ready_even);
   }
-  // epilogue: O / l and the log-sum-exp
+  // epilogue: O / l and the log-sum-exp (a row that sees no key tile: O = 0,
+  // LSE = -inf, and tensor memory holds no product to read)
   if (ok && warp_wait(&io.o_final[t], 0, wc)) {
     tc_fence_after();
     const bool valid = n < io.N;
-    const float inv_l = __frcp_rn(l);        // reciprocal without the division slow-path call
+    const bool empty = kSparse && io.n_act == 0;
+    const float inv_l = empty ? 0.f : __frcp_rn(l);   // reciprocal without the division slow-path call
     const size_t row_off = (static_cast<size_t>(pr.bh) * io.N + n) * kHeadDim;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t o[32];
       tmem_ld32(tO + q * 32, o);
       tmem_ld_wait(o);
+      if (kSparse && empty) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
       if (valid) {
         if (io.out_f32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(io.out) + row_off + q * 32);
@@ -213,7 +222,8 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
       }
     }
     if (valid && io.lse != nullptr) {
-      io.lse[static_cast<size_t>(pr.bh) * io.N + n] = (m_used * c + lg2_approx(l)) * 0.69314718055994530942f;
+      io.lse[static_cast<size_t>(pr.bh) * io.N + n] =
+          empty ? -INFINITY : (m_used * c + lg2_approx(l)) * 0.69314718055994530942f;
     }
   }
 }

@@ -51,6 +51,7 @@ constexpr int kProWarps = 6;                       // in-loop operand warps per 
 constexpr int kProThreads = kProWarps * 32;
 constexpr int kQRotThreads = 14 * 32;              // warps 2-15 rotate Q
 constexpr int kBarQRot = 1;                        // named barrier of the Q rotation
+constexpr int kMaxKvTiles = 4096;                  // block-sparse launches: N <= 4096 x 128 keys
 // Register split of the 4 x 128 x 128 launch registers between warpgroups:
 // producer / MMA warpgroup, the two softmax warpgroups, the operand warpgroup.
 constexpr uint32_t kIssueRegs = 80;
@@ -71,6 +72,8 @@ struct __align__(1024) Smem {
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
+  int n_act;                                           // key tiles this pair attends to
+  // block-sparse launches: the tiles' indices (uint16_t[kMaxKvTiles]) follow the struct
 };
 
 struct Params {
@@ -79,6 +82,7 @@ struct Params {
   void* out;
   float* lse;
   int* status;
+  const uint8_t* kv_mask;   // [B*H][clusters][n_kv] block mask, or nullptr (all key tiles)
   int N;
   int n_kv;
   int clusters;       // CTA pairs per (b, h): 512 query rows each
@@ -87,6 +91,39 @@ struct Params {
   int convert_v;      // convert V halves bf16 -> fp16 in the loop
   float scale_log2;   // log2(e) / sqrt(D)
 };
+
+// Block-sparse launches keep the pair's list of key tiles right after Smem.
+__device__ __forceinline__ uint16_t* kv_list(Smem& sm) { return reinterpret_cast<uint16_t*>(&sm + 1); }
+__device__ __forceinline__ const uint16_t* kv_list(const Smem& sm) {
+  return reinterpret_cast<const uint16_t*>(&sm + 1);
+}
+
+// Key tile visited at step i: the i-th tile of the pair's list (kSparse),
+// else tile i.  Number of steps: the list's length, else all n_kv tiles.
+template <bool kSparse>
+__device__ __forceinline__ int kv_tile(const Smem& sm, int i) {
+  return kSparse ? static_cast<int>(kv_list(sm)[i]) : i;
+}
+template <bool kSparse>
+__device__ __forceinline__ int kv_steps(const Smem& sm, const Params& p) {
+  return kSparse ? sm.n_act : p.n_kv;
+}
+
+// Compact the pair's row of the block mask into the tile list and n_act (one
+// warp; both CTAs of the pair read the same row).
+__device__ __forceinline__ void build_kv_list(Smem& sm, const Params& p, const Pair& pr, int qblock, int lane) {
+  const uint8_t* row = p.kv_mask + (static_cast<size_t>(pr.bh) * p.clusters + qblock) * p.n_kv;
+  uint16_t* list = kv_list(sm);
+  int count = 0;
+  for (int base = 0; base < p.n_kv; base += 32) {
+    const int tile = base + lane;
+    const bool on = tile < p.n_kv && row[tile] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, on);
+    if (on) list[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(tile);
+    count += __popc(bal);
+  }
+  if (lane == 0) sm.n_act = count;
+}
 
 // Q tile chunk c (0..2047): byte offset in the 128B-swizzled layout of two
 // 128-row x 64-channel boxes, its row and first channel.
@@ -167,7 +204,7 @@ __device__ __forceinline__ void convert_half_f16(uint8_t* tile, int pt) {
 // kPrepared: K / V halves land MMA-ready; their bytes are counted on the even
 // CTA's barriers (one expect_tx there covers both halves).  Otherwise each
 // CTA counts its own halves locally for its operand warps.
-template <bool kPrepared>
+template <bool kPrepared, bool kSparse>
 __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const CUtensorMap* tm_q,
                                               const CUtensorMap* tm_k, const CUtensorMap* tm_v, const Pair& pr,
                                               const WaitCtx& wc) {
@@ -180,10 +217,11 @@ __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const C
       tma_load_3d(sm.q[t] + b * kQBoxBytes, tm_q, &sm.q_full, b * 64, pr.row0[t], pr.bh);
   const bool leader = pr.rank == 0;
   int issued = 0;
-  for (int j = 0; j < p.n_kv; ++j) {
+  const int steps = kv_steps<kSparse>(sm, p);
+  for (int j = 0; j < steps; ++j) {
     const int s = j % kStages;
     const uint32_t ph = (j / kStages) & 1;
-    const int key0 = j * kTile;
+    const int key0 = kv_tile<kSparse>(sm, j) * kTile;
     if (!mbar_wait(&sm.kv_empty[s], ph ^ 1, wc)) break;
     if (kPrepared) {
       if (leader) mbar_arrive_expect_tx(&sm.k_full[s], 2 * kKHalfBytes);
@@ -227,7 +265,7 @@ __device__ __forceinline__ void producer_role(Smem& sm, const Params& p, const C
 // ---------------------------------------------------------------- MMA issuer
 // Even CTA only.  Completion of pair MMAs is signalled to the barrier of the
 // same name in both CTAs.
-template <bool kPrepared>
+template <bool kPrepared, bool kSparse>
 __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tmem, const WaitCtx& wc) {
   constexpr uint32_t idesc_qk = instr_desc(1, 1, 256, 128, 0, 0);   // bf16 x bf16, both K-major
   constexpr uint32_t idesc_pv = instr_desc(0, 0, 256, 128, 0, 1);   // f16 x f16, V MN-major
@@ -242,7 +280,8 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
   uint64_t* v_bar = kPrepared ? sm.v_full : sm.v_ready;
   bool ok = mbar_wait(&sm.q_ready, 0, wc);
   tc_fence_after();
-  for (int j = 0; ok && j <= p.n_kv; ++j) {
+  const int n_act = kv_steps<kSparse>(sm, p);
+  for (int j = 0; ok && j <= n_act; ++j) {
     const int s = j % kStages;
     const int sp = (j + kStages - 1) % kStages;
 #pragma unroll
@@ -258,9 +297,9 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
         mma_ts_pair(tO, tS, vd, idesc_pv, j > 1 ? 1u : 0u);
 #pragma unroll
         for (int kk = 1; kk < 8; ++kk) mma_ts_pair(tO, tS + kk * 8, vd + kk * (2048 >> 4), idesc_pv, 1u);
-        if (j == p.n_kv) commit_both(&sm.o_final[t]);
+        if (j == n_act) commit_both(&sm.o_final[t]);
       }
-      if (j < p.n_kv) {
+      if (j < n_act) {
         // S_t = Q_t K_j^T
         if (t == 0) {
           if (!(ok = mbar_wait(&k_bar[s], (j / kStages) & 1, wc))) break;
@@ -280,6 +319,10 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
     if (!ok) break;
     // one release per stage: the commit tracks Q K_{j-1}^T and P V_{j-1}
     if (j > 0) commit_both(&sm.kv_empty[sp]);
+  }
+  if (kSparse && ok && n_act == 0) {   // no key tile: nothing to wait for
+    commit_both(&sm.o_final[0]);
+    commit_both(&sm.o_final[1]);
   }
   // every MMA issued above has completed once this arrives
   tc_commit_pair(cl(&sm.mma_drain, 0));
@@ -304,15 +347,18 @@ __device__ __forceinline__ void rotate_q(Smem& sm, const Params& p, const Pair& 
 }
 
 // In-loop operand work (warps 2-3, 12-15) on this CTA's K_j and V_j halves.
+template <bool kSparse>
 __device__ __forceinline__ void kv_prologue_role(Smem& sm, const Params& p, const Pair& pr, int warp, int lane,
                                                  const WaitCtx& wc) {
   const int pt = (warp < 4 ? (warp - 2) * 32 : 64 + (warp - 12) * 32) + lane;
-  for (int j = 0; j < p.n_kv; ++j) {
+  const int steps = kv_steps<kSparse>(sm, p);
+  for (int j = 0; j < steps; ++j) {
     const int s = j % kStages;
     const uint32_t ph = (j / kStages) & 1;
     if (!warp_wait(&sm.k_full[s], ph, wc)) break;
     if (p.rotate_k)
-      rotate_chunks<kKHalfBytes / 16, kProThreads, 2, true>(sm.k[s], j * kTile + 64 * static_cast<int>(pr.rank),
+      rotate_chunks<kKHalfBytes / 16, kProThreads, 2, true>(sm.k[s],
+                                                            kv_tile<kSparse>(sm, j) * kTile + 64 * static_cast<int>(pr.rank),
                                                             p, pt);
     fence_proxy_async_smem();
     __syncwarp();
@@ -325,7 +371,7 @@ __device__ __forceinline__ void kv_prologue_role(Smem& sm, const Params& p, cons
   }
 }
 
-template <bool kPrepared>
+template <bool kPrepared, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -365,8 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
+  if (kSparse && warp == 2) build_kv_list(sm, p, pr, cluster % p.clusters, lane);
   tc_fence_before();
-  cluster_sync();          // both CTAs' barriers initialised, tensor memory allocated
+  cluster_sync();          // both CTAs' barriers initialised, tensor memory allocated, key list built
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wc{&sm.abort, p.status, cl(&sm.abort, pr.peer)};
@@ -376,20 +423,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_increase<kSoftmaxRegs>();
     rotate_q<4>(sm, p, pr, warp, lane, wc);
     attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.n_kv, p.out_f32, p.scale_log2,
-                       nullptr, nullptr, 0};
-    attn::softmax_slot<false>(io, tmem, pr, warp, lane, wc);
+                       nullptr, nullptr, 0, kv_list(sm), kv_steps<kSparse>(sm, p)};
+    attn::softmax_slot<false, kSparse>(io, tmem, pr, warp, lane, wc);
   } else {
     if (wg == 0)
       regs_decrease<kIssueRegs>();
     else
       regs_decrease<kOperandRegs>();
     if (warp == 0) {
-      if (lane == 0) producer_role<kPrepared>(sm, p, &tm_q, &tm_k, &tm_v, pr, wc);
+      if (lane == 0) producer_role<kPrepared, kSparse>(sm, p, &tm_q, &tm_k, &tm_v, pr, wc);
     } else if (warp == 1) {
-      if (lane == 0 && pr.rank == 0) mma_role<kPrepared>(sm, p, tmem, wc);
+      if (lane == 0 && pr.rank == 0) mma_role<kPrepared, kSparse>(sm, p, tmem, wc);
     } else {
       rotate_q<2>(sm, p, pr, warp, lane, wc);
-      if (!kPrepared) kv_prologue_role(sm, p, pr, warp, lane, wc);
+      if (!kPrepared) kv_prologue_role<kSparse>(sm, p, pr, warp, lane, wc);
     }
   }
 
@@ -416,15 +463,15 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, bool f16, int b
   return r == CUDA_SUCCESS;
 }
 
-template <bool kPrepared>
+template <bool kPrepared, bool kSparse>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, long long grid,
            cudaStream_t s) {
-  const size_t smem = sizeof(Smem) + 1024;
+  const size_t smem = sizeof(Smem) + (kSparse ? kMaxKvTiles * sizeof(uint16_t) : 0) + 1024;
   static thread_local int configured_device = -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -4;
   if (configured_device != dev) {
-    if (cudaFuncSetAttribute(attn_fwd_bf16_kernel<kPrepared>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_bf16_kernel<kPrepared, kSparse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return -4;
     configured_device = dev;
@@ -441,7 +488,7 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<kPrepared>, mq, mk, mv, p) == cudaSuccess ? 0 : -4;
+  return cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<kPrepared, kSparse>, mq, mk, mv, p) == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace
@@ -459,8 +506,10 @@ int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   p.lse = a.lse;
   p.status = device_status_word();
   if (p.status == nullptr) return -4;
+  p.kv_mask = a.kv_mask;
   p.N = a.N;
   p.n_kv = (a.N + kTile - 1) / kTile;
+  if (a.kv_mask != nullptr && p.n_kv > kMaxKvTiles) return -2;
   p.clusters = (a.N + 4 * kTile - 1) / (4 * kTile);
   p.out_f32 = a.out_f32 ? 1 : 0;
   p.rotate_k = (a.cos != nullptr && !a.k_rotated) ? 1 : 0;
@@ -468,8 +517,10 @@ int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kHeadDim));
   const long long grid = 2LL * BH * p.clusters;
   if (grid > 0x7FFFFFFFLL) return -1;
-  if (!p.rotate_k && !p.convert_v) return launch<true>(mq, mk, mv, p, grid, s);
-  return launch<false>(mq, mk, mv, p, grid, s);
+  const bool prepared = !p.rotate_k && !p.convert_v;
+  if (a.kv_mask != nullptr)
+    return prepared ? launch<true, true>(mq, mk, mv, p, grid, s) : launch<false, true>(mq, mk, mv, p, grid, s);
+  return prepared ? launch<true, false>(mq, mk, mv, p, grid, s) : launch<false, false>(mq, mk, mv, p, grid, s);
 }
 
 }  // namespace dit

@@ -108,9 +108,14 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
   return cuda_status(dit::launch_prepare_kv(a, static_cast<cudaStream_t>(stream)));
 }
 
-int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
-                     void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
-                     dit_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks and launch shared by the dense and block-sparse entries.
+int forward_bf16(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                 const uint8_t* kv_mask, void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                 dit_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N_txt < 0 || N_img < 0) return DIT_ERR_INVALID_ARG;
@@ -120,12 +125,30 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
   if (D != 128) return DIT_ERR_UNSUPPORTED;
   if ((dtype & ~(DIT_OUT_F32 | DIT_K_ROTATED | DIT_V_F16)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
   if ((dtype & DIT_K_ROTATED) && rope_cos == nullptr) return DIT_ERR_INVALID_ARG;
+  if (kv_mask != nullptr && N > static_cast<long long>(DIT_SPARSE_MAX_KV_TILES) * 128) return DIT_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIT_ERR_MISALIGNED;
   if ((rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) || (lse != nullptr && !aligned4(lse)))
     return DIT_ERR_MISALIGNED;
   dit::AttnFwdArgs a{q,   k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N), (dtype & DIT_OUT_F32) != 0,
-                     (dtype & DIT_K_ROTATED) != 0, (dtype & DIT_V_F16) != 0};
+                     (dtype & DIT_K_ROTATED) != 0, (dtype & DIT_V_F16) != 0, kv_mask};
   return launcher_status(dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                     void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                     dit_stream_t stream) {
+  return forward_bf16(q, k, v, rope_cos, rope_sin, nullptr, out, lse, B, H, N_txt, N_img, D, dtype, stream);
+}
+
+int dit_attn_forward_sparse(const void* q, const void* k, const void* v, const float* rope_cos,
+                            const float* rope_sin, const uint8_t* kv_mask, void* out, float* lse, int B, int H,
+                            int N_txt, int N_img, int D, int dtype, dit_stream_t stream) {
+  if (kv_mask == nullptr) return DIT_ERR_INVALID_ARG;
+  return forward_bf16(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, B, H, N_txt, N_img, D, dtype, stream);
 }
 
 int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float* rope_sin, uint8_t* x_fp8,

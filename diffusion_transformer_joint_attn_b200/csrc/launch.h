@@ -63,6 +63,7 @@ struct AttnFwdArgs {
   bool out_f32;
   bool k_rotated;   // k already carries the rotary embedding: rotate q only
   bool v_f16;       // v is given as fp16 (otherwise bf16)
+  const uint8_t* kv_mask = nullptr;   // [B*H][ceil(N/512)][ceil(N/128)] block mask, or nullptr (dense)
 };
 struct AttnFwdFp8Args {
   const void* q8;      // e4m3 [B][H][N][128]

@@ -58,6 +58,7 @@ typedef enum { DIT_BF16 = 0, DIT_FP8_E4M3 = 1 } dit_dtype_t;
 #define DIT_K_ROTATED 0x200 /* k already carries the rotary embedding (dit_rope_apply); rotate q only */
 #define DIT_V_F16 0x400     /* v is given as fp16 (dit_attn_prepare_kv) instead of bf16 */
 #define DIT_PART_F32 0x800  /* dit_attn_merge: the part outputs are fp32 instead of bf16 */
+#define DIT_SPARSE_MAX_KV_TILES 4096  /* dit_attn_forward_sparse: N <= 4096 x 128 keys */
 #define DIT_MERGE_MAX_PARTS 16
 
 /*
@@ -152,6 +153,31 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                      void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
                      dit_stream_t stream);
+
+/*
+ * dit_attn_forward_sparse — dit_attn_forward restricted to the key tiles a
+ * block mask selects, skipping the others entirely (no load, no product, no
+ * exponential).  The pages name sparse attention only as prior art
+ * (Sol-Attention and VC-Attention on B200: scopeai.cc, section on the effect
+ * of each optimisation) and give no rule for choosing tiles, so the mask is an
+ * input.
+ *
+ *   kv_mask   device uint8 [B][H][ceil(N/512)][ceil(N/128)]: query row n of
+ *             (b, h) attends to key m only where
+ *             kv_mask[b][h][n / 512][m / 128] is nonzero (512-row query
+ *             blocks x 128-key tiles, the kernel's units of work).  A row
+ *             whose block selects no tile gets out = 0 and lse = -inf (the
+ *             sum over an empty key set), which dit_attn_merge treats as an
+ *             empty part.
+ *   N         at most DIT_SPARSE_MAX_KV_TILES x 128, else
+ *             DIT_ERR_UNSUPPORTED.
+ * Everything else (arguments, dtype flags, alignment, status) as
+ * dit_attn_forward; an all-ones mask gives dit_attn_forward's result bit for
+ * bit.
+ */
+int dit_attn_forward_sparse(const void* q, const void* k, const void* v, const float* rope_cos,
+                            const float* rope_sin, const uint8_t* kv_mask, void* out, float* lse, int B, int H,
+                            int N_txt, int N_img, int D, int dtype, dit_stream_t stream);
 
 /*
  * dit_attn_quantize_fp8 — FP8 E4M3 operands for dit_attn_forward_fp8.

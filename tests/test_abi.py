@@ -71,6 +71,19 @@ def test_forward_argument_errors(lib):
     assert _fwd(lib, lse=0x70002) == dit.DIT_ERR_MISALIGNED
 
 
+def test_sparse_forward_argument_errors(lib):
+    f = lib.dit_attn_forward_sparse
+
+    def call(mask=0x9000, nt=8, ni=8, q=0x10000, D=128, dtype=0):
+        return f(q, 0x20000, 0x30000, None, None, mask, 0x40000, None, 1, 1, nt, ni, D, dtype, None)
+    assert call(mask=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(nt=0, ni=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=dit.DIT_FP8_E4M3) == dit.DIT_ERR_UNSUPPORTED
+    assert call(nt=0, ni=dit.DIT_SPARSE_MAX_KV_TILES * 128 + 1) == dit.DIT_ERR_UNSUPPORTED
+    assert call(q=0x10008) == dit.DIT_ERR_MISALIGNED
+
+
 def test_rope_table_argument_errors(lib):
     ax = (ctypes.c_int32 * 3)(16, 56, 56)
     bad = (ctypes.c_int32 * 3)(16, 55, 57)
