@@ -124,8 +124,12 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
   if (kScaled && n < io.N) qs = __ldg(io.q_scale + n / 64);
   float m_used = 0.f, l = 0.f;
   bool ok = true;
+  // the list is ascending, so the ragged last tile can only be its last entry
+  const bool last_is_tail = !kSparse || (io.n_act > 0 && io.kv_list[io.n_act - 1] == io.n_kv - 1);
   for (int i = 0; i < io.n_act; ++i) {
-    const int j = kSparse ? static_cast<int>(io.kv_list[i]) : i;   // key tile
+    // key tile (read from the list only where the FP8 block scales need it)
+    const int j = (kSparse && kScaled) ? static_cast<int>(io.kv_list[i]) : i;
+    const bool tail_step = kSparse ? (i == io.n_act - 1 && last_is_tail) : (j == io.n_kv - 1);
     float sc0 = 1.0f, sc1 = 1.0f;
     if (kScaled) {
       const float ks0 = __ldg(io.k_scale + 2 * j);
@@ -141,7 +145,7 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
 #pragma unroll
     for (int q = 0; q < 4; ++q) tmem_ld_wait(s + q * 32);
     float* f = reinterpret_cast<float*>(s);
-    if (j == io.n_kv - 1 && last_valid < kTile) {     // keys past N in the last tile
+    if (tail_step && last_valid < kTile) {            // keys past N in the last tile
 #pragma unroll
       for (int e = 0; e < 128; ++e)
         if (e >= last_valid) f[e] = -INFINITY;

@@ -230,3 +230,17 @@ def test_reruns_are_bitwise_identical():
 
 def test_status_word_is_clear():
     assert dit.dit_attn_get_status() == dit.DIT_OK
+
+
+def test_ulysses_single_rank_runs_the_library_kernel():
+    """With one rank the Ulysses exchanges are the identity and the call is
+    the library's forward on prepared operands (bit-identical to the plain
+    forward)."""
+    from diffusion_transformer_joint_attn_b200 import ulysses
+    w = W.WORKLOADS["tiny_256"]
+    _, _, _, qd, kd, vd = device_inputs(w)
+    c, s = dit.rope_table(torch.from_numpy(W.positions(w)).cuda())
+    a, la = ulysses.ulysses_attention(qd, kd, vd, c, s, n_txt=w.n_txt)
+    b, lb = dit.forward(qd, kd, vd, c, s, n_txt=w.n_txt)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
