@@ -38,6 +38,7 @@ WORKLOAD = "t2i_2048px"
 METRIC = "joint-attention TFLOP/s and % of B200 dense BF16/FP8 tensor peak (1 GPU)"
 UNIT = "TFLOP/s"
 FALLBACK_PEAK_BF16 = 1590.0
+E2E_CHUNK_HEADS = 4          # heads per chunk of the host-buffer pipeline
 
 
 # ------------------------------------------------------------------ multi-rank
@@ -413,22 +414,27 @@ def run_native(args):
     merge = time_merge(args, w, lib, out, lse, stream, dev)
     sparse = time_sparse(args, w, lib, q, k_rot, v_f16, cos, sin, out, lse, stream, dev, kern_ms)
 
-    # end to end through the public API: pinned host inputs in, O and LSE out
+    # end to end through the public C ABI with host buffers: pinned q, k, v
+    # and positions in, O and LSE out; dit_attn_forward_host moves chunks of
+    # E2E_CHUNK_HEADS heads through a device workspace, overlapping its copies
+    # with the kernels
     q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     pos_p = pos_h.pin_memory()
     out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (q_p, k_p, v_p, pos_p))
     d2h = out_p.numel() * out_p.element_size() + lse_p.numel() * lse_p.element_size()
+    ws_bytes = lib.dit_attn_forward_host_workspace(w.B, w.H, w.N, w.D, dit.DIT_BF16, E2E_CHUNK_HEADS)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        q.copy_(q_p, non_blocking=True)
-        k.copy_(k_p, non_blocking=True)
-        v.copy_(v_p, non_blocking=True)
         pos.copy_(pos_p, non_blocking=True)
-        step()
-        out_p.copy_(out, non_blocking=True)
-        lse_p.copy_(lse, non_blocking=True)
+        assert lib.dit_rope_table_build(pos.data_ptr(), w.N, w.D, axes, W.ROPE_THETA, cos.data_ptr(),
+                                        sin.data_ptr(), s_ptr) == 0
+        assert lib.dit_attn_forward_host(q_p.data_ptr(), k_p.data_ptr(), v_p.data_ptr(), cos.data_ptr(),
+                                         sin.data_ptr(), out_p.data_ptr(), lse_p.data_ptr(), w.B, w.H, w.n_txt,
+                                         w.n_img, w.D, dit.DIT_BF16, workspace.data_ptr(), ws_bytes,
+                                         E2E_CHUNK_HEADS, s_ptr) == 0
 
     for _ in range(min(args.warmup, 3)):
         e2e_step()
@@ -473,7 +479,8 @@ def run_native(args):
                          "kernel": "attn_fwd_bf16_kernel", "peak_source": peak_src,
                          "kernel_ms": kern_ms},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms / e2e_steps},
+                    "ms_per_step": e2e_ms / e2e_steps,
+                    "api": "dit_attn_forward_host, %d heads per chunk, pinned host buffers" % E2E_CHUNK_HEADS},
             "gpu_launches": 3 * args.steps,
             "fp8": fp8,
             "merge": merge,

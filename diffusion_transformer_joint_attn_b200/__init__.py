@@ -134,6 +134,38 @@ def _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dty
                      tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
 
 
+def dit_attn_forward_host_workspace(B: int, H: int, N: int, dtype: int = DIT_BF16, chunk_heads: int = 4) -> int:
+    """Device workspace bytes dit_attn_forward_host needs (0 for invalid arguments)."""
+    return int(load_library().dit_attn_forward_host_workspace(B, H, N, 128, dtype, chunk_heads))
+
+
+def dit_attn_forward_host(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: int, workspace,
+                          dtype: int = DIT_BF16, chunk_heads: int = 4, stream=None) -> None:
+    """out, lse (CPU tensors) <- joint attention of CPU bf16 q, k, v [B, H, N, D]; the tables and the
+    workspace (uint8) are CUDA tensors.  Pinned CPU tensors let the copies overlap the kernels."""
+    import torch
+    _require(q.dim() == 4 and q.shape == k.shape == v.shape, "q, k, v must share one [B, H, N, D] shape")
+    B, H, N, D = q.shape
+    _require(N == n_txt + n_img, "N must equal n_txt + n_img")
+    for t in (q, k, v):
+        _require(not t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "q, k, v must be contiguous CPU bf16")
+    out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
+    _require(not out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q.shape,
+             "out must be a contiguous CPU tensor of q's shape and the requested dtype")
+    if lse is not None:
+        _require(not lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and
+                 tuple(lse.shape) == (B, H, N), "lse must be a contiguous CPU fp32 [B, H, N] tensor")
+    if rope_cos is not None or rope_sin is not None:
+        for t in (rope_cos, rope_sin):
+            _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _require(workspace.is_cuda and workspace.is_contiguous(), "workspace must be a contiguous CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load_library().dit_attn_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(out),
+                                                _ptr(lse), B, H, n_txt, n_img, D, dtype, _ptr(workspace), nbytes,
+                                                chunk_heads, _stream(stream)), "dit_attn_forward_host")
+
+
 def dit_attn_forward_sparse(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, n_txt: int, n_img: int,
                             dtype: int = DIT_BF16, stream=None) -> None:
     """dit_attn_forward restricted to the key tiles of kv_mask (CUDA uint8
@@ -267,6 +299,25 @@ def merge(o_parts, lse_parts, out_f32: bool = False, with_lse: bool = True, stre
     lse = torch.empty(o0.shape[:3], dtype=torch.float32, device=o0.device) if with_lse else None
     flags = (DIT_PART_F32 if o0.dtype == torch.float32 else 0) | (DIT_OUT_F32 if out_f32 else 0)
     dit_attn_merge(o_parts, lse_parts, out, lse, DIT_BF16 | flags, stream)
+    return out, lse
+
+
+def forward_host(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool = False,
+                 with_lse: bool = True, chunk_heads: int = 4, workspace=None, pin: bool = True, stream=None):
+    """Attention of CPU q, k, v through dit_attn_forward_host; allocates (pinned) CPU outputs and, if none is
+    given, the device workspace.  Returns (out, lse) once the results are on the host."""
+    import torch
+    B, H, N, D = q.shape
+    out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, pin_memory=pin)
+    lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=pin) if with_lse else None
+    dtype = DIT_BF16 | (DIT_OUT_F32 if out_f32 else 0)
+    if workspace is None:
+        nbytes = dit_attn_forward_host_workspace(B, H, N, dtype, chunk_heads)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    dit_attn_forward_host(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt, workspace, dtype, chunk_heads,
+                          stream)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    s.synchronize()
     return out, lse
 
 

@@ -144,6 +144,33 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
   return forward_bf16(q, k, v, rope_cos, rope_sin, nullptr, out, lse, B, H, N_txt, N_img, D, dtype, stream);
 }
 
+size_t dit_attn_forward_host_workspace(int B, int H, int N, int D, int dtype, int chunk_heads) {
+  if (B < 1 || H < 1 || N < 1 || chunk_heads < 1 || D != 128) return 0;
+  if ((dtype & ~DIT_OUT_F32) != DIT_BF16) return 0;
+  return dit::host_forward_workspace_bytes(B * H, N, chunk_heads, (dtype & DIT_OUT_F32) != 0);
+}
+
+int dit_attn_forward_host(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                          void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                          void* workspace, size_t workspace_bytes, int chunk_heads, dit_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || workspace == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N_txt < 0 || N_img < 0 || chunk_heads < 1) return DIT_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img;
+  if (N < 1 || N > 0x7FFFFFFF || static_cast<long long>(B) * H > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if ((dtype & ~DIT_OUT_F32) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+  const bool out_f32 = (dtype & DIT_OUT_F32) != 0;
+  if (workspace_bytes < dit::host_forward_workspace_bytes(B * H, static_cast<int>(N), chunk_heads, out_f32))
+    return DIT_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || (rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))))
+    return DIT_ERR_MISALIGNED;
+  dit::HostForwardArgs a{q, k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N), out_f32, workspace,
+                         chunk_heads};
+  return cuda_status(dit::host_forward(a, static_cast<cudaStream_t>(stream)));
+}
+
 int dit_attn_forward_sparse(const void* q, const void* k, const void* v, const float* rope_cos,
                             const float* rope_sin, const uint8_t* kv_mask, void* out, float* lse, int B, int H,
                             int N_txt, int N_img, int D, int dtype, dit_stream_t stream) {

@@ -1,0 +1,165 @@
+// Attention on q, k, v that live in host memory: the library moves them
+// through a caller-provided device workspace in chunks of heads, with the
+// host-to-device copies, the kernels and the device-to-host copies of
+// consecutive chunks overlapping (two workspace buffers, two copy streams,
+// the kernels on the caller's stream).  With pinned host memory the step
+// then takes about as long as the larger of its copies, not their sum.
+#include <algorithm>
+#include <mutex>
+
+#include "launch.h"
+
+namespace dit {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kBuffers = 2;
+
+// Copy streams and the events that order one buffer's chunk: loaded (host to
+// device done), computed (kernels done), stored (device to host done).
+struct CopyEngines {
+  bool ready = false;
+  cudaStream_t h2d = nullptr;
+  cudaStream_t d2h = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t loaded[kBuffers] = {};
+  cudaEvent_t computed[kBuffers] = {};
+  cudaEvent_t stored[kBuffers] = {};
+};
+CopyEngines g_engines[kMaxDevices];
+std::mutex g_mu;   // one enqueue sequence at a time (the events are shared)
+
+cudaError_t engines_for(int dev, CopyEngines** out) {
+  CopyEngines& e = g_engines[dev];
+  if (!e.ready) {
+    cudaError_t r = cudaStreamCreateWithFlags(&e.h2d, cudaStreamNonBlocking);
+    if (r == cudaSuccess) r = cudaStreamCreateWithFlags(&e.d2h, cudaStreamNonBlocking);
+    if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.start, cudaEventDisableTiming);
+    for (int b = 0; b < kBuffers && r == cudaSuccess; ++b) {
+      r = cudaEventCreateWithFlags(&e.loaded[b], cudaEventDisableTiming);
+      if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.computed[b], cudaEventDisableTiming);
+      if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.stored[b], cudaEventDisableTiming);
+    }
+    if (r != cudaSuccess) return r;
+    e.ready = true;
+  }
+  *out = &e;
+  return cudaSuccess;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// A launcher's dit status as a runtime error (the launch's own error if it
+// recorded one).
+cudaError_t launch_status(int rc) {
+  if (rc == 0) return cudaSuccess;
+  const cudaError_t e = cudaGetLastError();
+  return e != cudaSuccess ? e : cudaErrorInvalidValue;
+}
+
+// Offsets of one buffer's arrays for `heads` heads of N tokens.
+struct BufferLayout {
+  size_t q, k, v, k_rot, v16, out, lse, bytes;
+};
+BufferLayout buffer_layout(int heads, int N, bool out_f32) {
+  const size_t elems = static_cast<size_t>(heads) * N * 128;
+  BufferLayout L;
+  size_t o = 0;
+  L.q = o;
+  o += align256(elems * 2);
+  L.k = o;
+  o += align256(elems * 2);
+  L.v = o;
+  o += align256(elems * 2);
+  L.k_rot = o;
+  o += align256(elems * 2);
+  L.v16 = o;
+  o += align256(elems * 2);
+  L.out = o;
+  o += align256(elems * (out_f32 ? 4 : 2));
+  L.lse = o;
+  o += align256(static_cast<size_t>(heads) * N * 4);
+  L.bytes = o;
+  return L;
+}
+
+}  // namespace
+
+size_t host_forward_workspace_bytes(int BH, int N, int chunk_heads, bool out_f32) {
+  const int heads = std::min(chunk_heads, BH);
+  return kBuffers * buffer_layout(heads, N, out_f32).bytes;
+}
+
+cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t r = cudaGetDevice(&dev);
+  if (r != cudaSuccess) return r;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  CopyEngines* e = nullptr;
+  if ((r = engines_for(dev, &e)) != cudaSuccess) return r;
+
+  const int BH = a.B * a.H;
+  const int chunk = std::min(a.chunk_heads, BH);
+  const BufferLayout L = buffer_layout(chunk, a.N, a.out_f32);
+  const size_t head_elems = static_cast<size_t>(a.N) * 128;
+  const size_t out_esize = a.out_f32 ? 4 : 2;
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+
+  // work the caller queued before this call (e.g. the rotary tables, or an
+  // earlier use of the workspace) precedes every copy of this call
+  if ((r = cudaEventRecord(e->start, s)) != cudaSuccess) return r;
+  if ((r = cudaStreamWaitEvent(e->h2d, e->start, 0)) != cudaSuccess) return r;
+
+  const int n_chunks = (BH + chunk - 1) / chunk;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int b = c % kBuffers;
+    const int h0 = c * chunk;
+    const int hc = std::min(chunk, BH - h0);
+    uint8_t* base = ws + static_cast<size_t>(b) * L.bytes;
+    const size_t in_off = static_cast<size_t>(h0) * head_elems * 2;
+    const size_t in_bytes = static_cast<size_t>(hc) * head_elems * 2;
+    // the buffer's previous chunk (of this call or of the previous one) has left the device
+    if ((r = cudaStreamWaitEvent(e->h2d, e->stored[b], 0)) != cudaSuccess) return r;
+    const void* src[3] = {a.q, a.k, a.v};
+    const size_t dst[3] = {L.q, L.k, L.v};
+    for (int i = 0; i < 3; ++i) {
+      r = cudaMemcpyAsync(base + dst[i], static_cast<const uint8_t*>(src[i]) + in_off, in_bytes,
+                          cudaMemcpyHostToDevice, e->h2d);
+      if (r != cudaSuccess) return r;
+    }
+    if ((r = cudaEventRecord(e->loaded[b], e->h2d)) != cudaSuccess) return r;
+    if ((r = cudaStreamWaitEvent(s, e->loaded[b], 0)) != cudaSuccess) return r;
+
+    float* lse = a.lse != nullptr ? reinterpret_cast<float*>(base + L.lse) : nullptr;
+    if (a.cos != nullptr) {
+      PrepareKVArgs p{base + L.k, base + L.v, a.cos, a.sin, base + L.k_rot, base + L.v16, 1, hc, a.N, 128};
+      if ((r = launch_prepare_kv(p, s)) != cudaSuccess) return r;
+      AttnFwdArgs f{base + L.q, base + L.k_rot, base + L.v16, a.cos, a.sin, base + L.out, lse, 1, hc, a.N,
+                    a.out_f32, true, true};
+      if ((r = launch_status(launch_attn_fwd_bf16(f, s))) != cudaSuccess) return r;
+    } else {
+      AttnFwdArgs f{base + L.q, base + L.k, base + L.v, nullptr, nullptr, base + L.out, lse, 1, hc, a.N,
+                    a.out_f32, false, false};
+      if ((r = launch_status(launch_attn_fwd_bf16(f, s))) != cudaSuccess) return r;
+    }
+    if ((r = cudaEventRecord(e->computed[b], s)) != cudaSuccess) return r;
+    if ((r = cudaStreamWaitEvent(e->d2h, e->computed[b], 0)) != cudaSuccess) return r;
+    r = cudaMemcpyAsync(static_cast<uint8_t*>(a.out) + static_cast<size_t>(h0) * head_elems * out_esize,
+                        base + L.out, static_cast<size_t>(hc) * head_elems * out_esize, cudaMemcpyDeviceToHost,
+                        e->d2h);
+    if (r != cudaSuccess) return r;
+    if (a.lse != nullptr) {
+      r = cudaMemcpyAsync(a.lse + static_cast<size_t>(h0) * a.N, lse, static_cast<size_t>(hc) * a.N * 4,
+                          cudaMemcpyDeviceToHost, e->d2h);
+      if (r != cudaSuccess) return r;
+    }
+    if ((r = cudaEventRecord(e->stored[b], e->d2h)) != cudaSuccess) return r;
+  }
+  // the caller's stream completes only after the results are on the host
+  for (int b = 0; b < kBuffers; ++b)
+    if ((r = cudaStreamWaitEvent(s, e->stored[b], 0)) != cudaSuccess) return r;
+  return cudaSuccess;
+}
+
+}  // namespace dit

@@ -91,6 +91,24 @@ struct MergeArgs {
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 
+// Host-buffer forward (host_pipeline.cu): q, k, v, out, lse in host memory,
+// moved through `workspace` in chunks of chunk_heads (b, h) pairs.
+struct HostForwardArgs {
+  const void* q;       // host bf16 [B][H][N][128]
+  const void* k;
+  const void* v;
+  const float* cos;    // device tables [N][64] or nullptr
+  const float* sin;
+  void* out;           // host bf16 (fp32 if out_f32)
+  float* lse;          // host fp32 [B][H][N] or nullptr
+  int B, H, N;
+  bool out_f32;
+  void* workspace;     // device, host_forward_workspace_bytes(...)
+  int chunk_heads;
+};
+size_t host_forward_workspace_bytes(int BH, int N, int chunk_heads, bool out_f32);
+cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s);
+
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s);

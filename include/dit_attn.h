@@ -35,6 +35,7 @@
 #ifndef DIT_ATTN_H
 #define DIT_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -153,6 +154,42 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                      void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
                      dit_stream_t stream);
+
+/*
+ * dit_attn_forward_host — dit_attn_forward on q, k, v in HOST memory, with
+ * the results written to host memory: the library moves chunks of
+ * chunk_heads (b, h) pairs through `workspace`, overlapping the copies to the
+ * device, the kernels (K rotation and V conversion, then the forward) and the
+ * copies back for consecutive chunks.  With page-locked host buffers the call
+ * takes about as long as the larger of its two copy directions; pageable
+ * buffers work but copy synchronously.
+ *
+ *   q, k, v     host bf16 [B][H][N][D].  They are read asynchronously: keep
+ *               them unchanged until `stream` has been synchronised.
+ *   rope_cos, rope_sin
+ *               DEVICE fp32 [N][D/2] tables (dit_rope_table_build), or both
+ *               NULL for no rotary embedding.
+ *   out, lse    host [B][H][N][D] bf16 (fp32 with DIT_OUT_F32) and fp32
+ *               [B][H][N] (lse may be NULL); complete once `stream` has been
+ *               synchronised.
+ *   dtype       DIT_BF16, optionally | DIT_OUT_F32.
+ *   workspace   device memory of at least
+ *               dit_attn_forward_host_workspace(B, H, N, D, dtype,
+ *               chunk_heads) bytes, 16-byte aligned; owned by the caller.
+ *               Consecutive calls may share it (the library orders its
+ *               reuse); concurrent calls must not.
+ *   chunk_heads (b, h) pairs per chunk, >= 1 (smaller chunks start the
+ *               overlap sooner, larger ones launch fewer kernels).
+ * The kernels run on `stream`; the copies on two streams the library creates
+ * once per device, ordered after the work already queued on `stream`, and
+ * `stream` waits for the last copy back.  Same limits and status handling as
+ * dit_attn_forward; a workspace smaller than required is
+ * DIT_ERR_INVALID_ARG.
+ */
+size_t dit_attn_forward_host_workspace(int B, int H, int N, int D, int dtype, int chunk_heads);
+int dit_attn_forward_host(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                          void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                          void* workspace, size_t workspace_bytes, int chunk_heads, dit_stream_t stream);
 
 /*
  * dit_attn_forward_sparse — dit_attn_forward restricted to the key tiles a
