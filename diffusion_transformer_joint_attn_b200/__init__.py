@@ -19,6 +19,8 @@ DIT_ERR_UNSUPPORTED = -2
 DIT_ERR_MISALIGNED = -3
 DIT_ERR_CUDA = -4
 DIT_ERR_TIMEOUT = -5
+DIT_ERR_WORKSPACE = -6
+DIT_STATIC_WORKSPACE_BYTES = 32 << 20
 DIT_BF16 = 0
 DIT_FP8_E4M3 = 1
 DIT_OUT_F32 = 0x100

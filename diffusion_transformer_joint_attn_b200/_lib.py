@@ -21,6 +21,7 @@ SIGNATURES = {
     "dit_attn_forward_host_workspace": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "dit_attn_forward_host": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, ctypes.c_size_t,
                                    _I, _VP]),
+    "dit_attn_forward_host_static": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_sparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_quantize_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),

@@ -171,6 +171,22 @@ int dit_attn_forward_host(const void* q, const void* k, const void* v, const flo
   return cuda_status(dit::host_forward(a, static_cast<cudaStream_t>(stream)));
 }
 
+int dit_attn_forward_host_static(const void* q, const void* k, const void* v, const float* rope_cos,
+                                 const float* rope_sin, void* out, float* lse, int B, int H, int N_txt, int N_img,
+                                 int D, int dtype, int chunk_heads, dit_stream_t stream) {
+  const long long N = static_cast<long long>(N_txt) + N_img;
+  if (B >= 1 && H >= 1 && N >= 1 && N <= 0x7FFFFFFF && chunk_heads >= 1 && D == 128 &&
+      (dtype & ~DIT_OUT_F32) == DIT_BF16 &&
+      dit::host_forward_workspace_bytes(B * H, static_cast<int>(N), chunk_heads, (dtype & DIT_OUT_F32) != 0) >
+          DIT_STATIC_WORKSPACE_BYTES)
+    return DIT_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const int rc = cuda_status(dit::static_workspace(&ws));
+  if (rc != DIT_OK) return rc;
+  return dit_attn_forward_host(q, k, v, rope_cos, rope_sin, out, lse, B, H, N_txt, N_img, D, dtype, ws,
+                               DIT_STATIC_WORKSPACE_BYTES, chunk_heads, stream);
+}
+
 int dit_attn_forward_sparse(const void* q, const void* k, const void* v, const float* rope_cos,
                             const float* rope_sin, const uint8_t* kv_mask, void* out, float* lse, int B, int H,
                             int N_txt, int N_img, int D, int dtype, dit_stream_t stream) {
@@ -211,6 +227,7 @@ int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8
 }
 
 static_assert(DIT_MERGE_MAX_PARTS == dit::kMergeMaxParts, "part limit of the header and the kernel differ");
+static_assert(DIT_STATIC_WORKSPACE_BYTES == dit::kStaticWorkspaceBytes, "static workspace size differs");
 
 int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, int R, void* out, float* lse_out,
                    int B, int H, int N, int D, int dtype, dit_stream_t stream) {
@@ -264,6 +281,7 @@ const char* dit_attn_status_string(int status) {
     case DIT_ERR_MISALIGNED: return "pointer not aligned (16 bytes; 4 for lse)";
     case DIT_ERR_CUDA: return "CUDA runtime or driver call failed";
     case DIT_ERR_TIMEOUT: return "a device-side wait timed out";
+    case DIT_ERR_WORKSPACE: return "problem needs more workspace than the static workspace holds";
     default: return "unknown status";
   }
 }

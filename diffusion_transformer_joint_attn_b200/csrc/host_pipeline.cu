@@ -83,7 +83,31 @@ BufferLayout buffer_layout(int heads, int N, bool out_f32) {
   return L;
 }
 
+// Workspace of dit_attn_forward_host_static: one array in the library's
+// device image, shared by every call on a device.  Every byte of it is
+// written (by a copy or a kernel) before it is read, so nothing needs
+// clearing.
+__device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
+
 }  // namespace
+
+cudaError_t static_workspace(void** out) {
+  static void* cached[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t r = cudaGetDevice(&dev);
+  if (r != cudaSuccess) return r;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    // with device `dev` current: the array's address in this device's copy of the image
+    void* ptr = nullptr;
+    if ((r = cudaGetSymbolAddress(&ptr, g_static_workspace)) != cudaSuccess) return r;
+    cached[dev] = ptr;
+  }
+  *out = cached[dev];
+  return cudaSuccess;
+}
 
 size_t host_forward_workspace_bytes(int BH, int N, int chunk_heads, bool out_f32) {
   const int heads = std::min(chunk_heads, BH);

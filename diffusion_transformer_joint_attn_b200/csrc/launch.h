@@ -107,6 +107,10 @@ struct HostForwardArgs {
   int chunk_heads;
 };
 size_t host_forward_workspace_bytes(int BH, int N, int chunk_heads, bool out_f32);
+// The library's static workspace for dit_attn_forward_host_static: its device
+// address on the current device (looked up once per device).
+constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
+cudaError_t static_workspace(void** out);
 cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s);
 
 // Builds the tensor maps and launches the BF16 forward kernel.

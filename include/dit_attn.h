@@ -50,7 +50,8 @@ typedef enum {
   DIT_ERR_UNSUPPORTED = -2, /* D != 128, unknown dtype or flag */
   DIT_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned (4-byte for lse) */
   DIT_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (launch, tensor map) */
-  DIT_ERR_TIMEOUT = -5      /* a device-side wait gave up (read via dit_attn_get_status) */
+  DIT_ERR_TIMEOUT = -5,     /* a device-side wait gave up (read via dit_attn_get_status) */
+  DIT_ERR_WORKSPACE = -6    /* dit_attn_forward_host_static: the problem needs more than the static workspace */
 } dit_status_t;
 
 /* Element type of q/k/v, OR-able with the flags below. */
@@ -190,6 +191,31 @@ size_t dit_attn_forward_host_workspace(int B, int H, int N, int D, int dtype, in
 int dit_attn_forward_host(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                           void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
                           void* workspace, size_t workspace_bytes, int chunk_heads, dit_stream_t stream);
+
+/*
+ * dit_attn_forward_host_static — dit_attn_forward_host without a caller
+ * workspace: the library uses a device array of DIT_STATIC_WORKSPACE_BYTES
+ * that is part of its own device image, so the call allocates nothing.  It
+ * is meant for callers that cannot hand the library device memory of their
+ * own: code whose device memory is all owned by another runtime's pool or a
+ * fixed budget, or latency-critical loops in which an allocation (which may
+ * synchronise the device) is not acceptable.  The pages describe no such
+ * entry point; it has no counterpart there.
+ *
+ * Arguments, results and status handling as dit_attn_forward_host, minus the
+ * workspace.  When dit_attn_forward_host_workspace(B, H, N, D, dtype,
+ * chunk_heads) exceeds DIT_STATIC_WORKSPACE_BYTES the call returns
+ * DIT_ERR_WORKSPACE and does nothing (fewer heads per chunk need less).
+ * Every call on a device uses the same array: calls that could overlap (from
+ * several host threads, or on streams not ordered with each other) race on
+ * it and must be serialised by the caller.  The first call on each device
+ * looks the array's address up (and creates the copy streams); make that
+ * first call outside any stream capture.
+ */
+#define DIT_STATIC_WORKSPACE_BYTES (32u << 20)
+int dit_attn_forward_host_static(const void* q, const void* k, const void* v, const float* rope_cos,
+                                 const float* rope_sin, void* out, float* lse, int B, int H, int N_txt, int N_img,
+                                 int D, int dtype, int chunk_heads, dit_stream_t stream);
 
 /*
  * dit_attn_forward_sparse — dit_attn_forward restricted to the key tiles a

@@ -109,6 +109,14 @@ def test_host_forward_workspace_and_argument_errors(lib):
     assert call(ws=0x8008) == dit.DIT_ERR_MISALIGNED
 
 
+def test_static_workspace_entry_rejects_oversize_without_a_gpu(lib):
+    # the size check comes before any CUDA call: 2048x2048 in 4-head chunks needs ~208 MB of workspace
+    rc = lib.dit_attn_forward_host_static(0x1000, 0x2000, 0x3000, None, None, 0x4000, None, 1, 24, 512, 16384, 128,
+                                          0, 4, None)
+    assert rc == dit.DIT_ERR_WORKSPACE
+    assert dit.dit_attn_status_string(rc) == "problem needs more workspace than the static workspace holds"
+
+
 def test_rope_table_argument_errors(lib):
     ax = (ctypes.c_int32 * 3)(16, 56, 56)
     bad = (ctypes.c_int32 * 3)(16, 55, 57)
