@@ -1,7 +1,7 @@
 // Attention on q, k, v that live in host memory: the library moves them
 // through a caller-provided device workspace in chunks of heads, with the
 // host-to-device copies, the kernels and the device-to-host copies of
-// consecutive chunks overlapping (two workspace buffers, two copy streams,
+// consecutive chunks overlapping (three workspace buffers, two copy streams,
 // the kernels on the caller's stream).  With pinned host memory the step
 // then takes about as long as the larger of its copies, not their sum.
 #include <algorithm>
@@ -13,7 +13,10 @@ namespace dit {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kBuffers = 2;
+// Three buffers: while chunk c is copied in, chunk c-1 can be computing and
+// chunk c-2 copying out, so the copy-in stream never waits for a buffer when
+// compute + copy-out of a chunk take as long as its copy-in.
+constexpr int kBuffers = 3;
 
 // Copy streams and the events that order one buffer's chunk: loaded (host to
 // device done), computed (kernels done), stored (device to host done).
@@ -135,11 +138,20 @@ cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s) {
   if ((r = cudaEventRecord(e->start, s)) != cudaSuccess) return r;
   if ((r = cudaStreamWaitEvent(e->h2d, e->start, 0)) != cudaSuccess) return r;
 
-  const int n_chunks = (BH + chunk - 1) / chunk;
-  for (int c = 0; c < n_chunks; ++c) {
+  // chunks: one head first and one head last (the copy-in before the first
+  // kernel and the kernel + copy-out after the last copy-in are not hidden;
+  // small end chunks keep them short), `chunk` heads in between
+  const bool ramp = BH > 2 && chunk > 1;
+  int c = 0;
+  for (int h0 = 0; h0 < BH; ++c) {
+    int hc;
+    if (!ramp)
+      hc = std::min(chunk, BH - h0);
+    else if (h0 == 0 || h0 == BH - 1)
+      hc = 1;
+    else
+      hc = std::min(chunk, BH - 1 - h0);   // the last head is kept for the final chunk
     const int b = c % kBuffers;
-    const int h0 = c * chunk;
-    const int hc = std::min(chunk, BH - h0);
     uint8_t* base = ws + static_cast<size_t>(b) * L.bytes;
     const size_t in_off = static_cast<size_t>(h0) * head_elems * 2;
     const size_t in_bytes = static_cast<size_t>(hc) * head_elems * 2;
@@ -179,6 +191,7 @@ cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s) {
       if (r != cudaSuccess) return r;
     }
     if ((r = cudaEventRecord(e->stored[b], e->d2h)) != cudaSuccess) return r;
+    h0 += hc;
   }
   // the caller's stream completes only after the results are on the host
   for (int b = 0; b < kBuffers; ++b)

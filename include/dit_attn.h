@@ -179,8 +179,9 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
  *               chunk_heads) bytes, 16-byte aligned; owned by the caller.
  *               Consecutive calls may share it (the library orders its
  *               reuse); concurrent calls must not.
- *   chunk_heads (b, h) pairs per chunk, >= 1 (smaller chunks start the
- *               overlap sooner, larger ones launch fewer kernels).
+ *   chunk_heads at most this many (b, h) pairs per chunk, >= 1; the first
+ *               and the last chunk hold one pair, so that little is left
+ *               unoverlapped at either end.
  * The kernels run on `stream`; the copies on two streams the library creates
  * once per device, ordered after the work already queued on `stream`, and
  * `stream` waits for the last copy back.  Same limits and status handling as

@@ -89,12 +89,12 @@ def test_host_forward_workspace_and_argument_errors(lib):
     al = lambda x: (x + 255) // 256 * 256
     N = 1000
     one = 5 * al(4 * N * 128 * 2) + al(4 * N * 128 * 2) + al(4 * N * 4)      # q k v k_rot v16, bf16 out, lse
-    assert f(1, 24, N, 128, 0, 4) == 2 * one
-    assert f(1, 2, N, 128, 0, 4) == 2 * (5 * al(2 * N * 256) + al(2 * N * 256) + al(2 * N * 4))   # chunk <= B*H
-    assert f(1, 24, N, 128, dit.DIT_OUT_F32, 4) == 2 * (one - al(4 * N * 256) + al(4 * N * 512))
+    assert f(1, 24, N, 128, 0, 4) == 3 * one                               # three buffers
+    assert f(1, 2, N, 128, 0, 4) == 3 * (5 * al(2 * N * 256) + al(2 * N * 256) + al(2 * N * 4))   # chunk <= B*H
+    assert f(1, 24, N, 128, dit.DIT_OUT_F32, 4) == 3 * (one - al(4 * N * 256) + al(4 * N * 512))
     assert f(1, 24, N, 64, 0, 4) == 0 and f(1, 24, N, 128, 0, 0) == 0 and f(1, 24, N, 128, 1, 4) == 0
     g = lib.dit_attn_forward_host
-    ok = dict(q=0x1000, ws=0x8000, wsb=2 * one, chunk=4, D=128, dtype=0)
+    ok = dict(q=0x1000, ws=0x8000, wsb=3 * one, chunk=4, D=128, dtype=0)
 
     def call(**kw):
         a = dict(ok, **kw)
@@ -102,7 +102,7 @@ def test_host_forward_workspace_and_argument_errors(lib):
                  a["chunk"], None)
     assert call(q=None) == dit.DIT_ERR_INVALID_ARG
     assert call(ws=None) == dit.DIT_ERR_INVALID_ARG
-    assert call(wsb=2 * one - 1) == dit.DIT_ERR_INVALID_ARG
+    assert call(wsb=3 * one - 1) == dit.DIT_ERR_INVALID_ARG
     assert call(chunk=0) == dit.DIT_ERR_INVALID_ARG
     assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
     assert call(dtype=dit.DIT_K_ROTATED) == dit.DIT_ERR_UNSUPPORTED
@@ -110,7 +110,7 @@ def test_host_forward_workspace_and_argument_errors(lib):
 
 
 def test_static_workspace_entry_rejects_oversize_without_a_gpu(lib):
-    # the size check comes before any CUDA call: 2048x2048 in 4-head chunks needs ~208 MB of workspace
+    # the size check comes before any CUDA call: 2048x2048 in 4-head chunks needs ~312 MB of workspace
     rc = lib.dit_attn_forward_host_static(0x1000, 0x2000, 0x3000, None, None, 0x4000, None, 1, 24, 512, 16384, 128,
                                           0, 4, None)
     assert rc == dit.DIT_ERR_WORKSPACE

@@ -53,7 +53,7 @@ def test_static_workspace_entry_matches_caller_workspace_entry():
 
 def test_static_workspace_entry_rejects_what_does_not_fit():
     lib = dit.load_library()
-    w = W.WORKLOADS["t2i_2048px"]                  # N = 16896: 4-head chunks need about 208 MB
+    w = W.WORKLOADS["t2i_2048px"]                  # N = 16896: 4-head chunks need about 312 MB
     assert dit.dit_attn_forward_host_workspace(w.B, w.H, w.N, dit.DIT_BF16, 4) > dit.DIT_STATIC_WORKSPACE_BYTES
     q = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.bfloat16)
     rc = lib.dit_attn_forward_host_static(q.data_ptr(), q.data_ptr(), q.data_ptr(), None, None, q.data_ptr(), None,
