@@ -26,6 +26,7 @@ SIGNATURES = {
     "dit_attn_quantize_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    "dit_attn_wait_selftest": (_I, [ctypes.c_longlong, _VP]),
     "dit_attn_get_status": (_I, [ctypes.POINTER(ctypes.c_int), _VP]),
     "dit_attn_status_string": (ctypes.c_char_p, [_I]),
     "dit_attn_last_cuda_error": (_I, []),

@@ -253,6 +253,12 @@ int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, in
   return cuda_status(dit::launch_merge(a, static_cast<cudaStream_t>(stream)));
 }
 
+int dit_attn_wait_selftest(long long limit_ns, dit_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000LL) return DIT_ERR_INVALID_ARG;
+  return cuda_status(dit::launch_wait_selftest(static_cast<unsigned long long>(limit_ns),
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 int dit_attn_get_status(int* status_host, dit_stream_t stream) {
   if (status_host == nullptr) return DIT_ERR_INVALID_ARG;
   int* word = dit::device_status_word();

@@ -113,6 +113,9 @@ constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
 cudaError_t static_workspace(void** out);
 cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s);
 
+// Bounded-wait self-test (wait_selftest.cu).
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
+
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s);

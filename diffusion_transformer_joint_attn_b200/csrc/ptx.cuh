@@ -113,15 +113,16 @@ __device__ __forceinline__ void report_timeout(const WaitCtx& w) {
 
 // Wait for the phase of `bar` with the given parity.  Returns false (and
 // leaves the phase unconsumed) if the CTA is aborting or the wait exceeded
-// kWaitLimitNs, which it reports.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+// limit_ns (kWaitLimitNs in the kernels), which it reports.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 15) == 0) {
       if (*w.abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         report_timeout(w);
         return false;
       }

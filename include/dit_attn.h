@@ -320,6 +320,17 @@ int dit_attn_merge(const void* const* o_parts, const float* const* lse_parts, in
                    int B, int H, int N, int D, int dtype, dit_stream_t stream);
 
 /*
+ * dit_attn_wait_selftest — exercise the bounded device-side waits that every
+ * kernel of the library uses: a one-thread kernel waits for a barrier phase
+ * that nothing completes, gives up after limit_ns nanoseconds
+ * (1 us .. 1 s), records DIT_ERR_TIMEOUT in the status word and returns.
+ * dit_attn_get_status then reports (and clears) DIT_ERR_TIMEOUT; the CUDA
+ * context stays usable.  Returns DIT_OK once launched, DIT_ERR_INVALID_ARG
+ * for a limit outside the range.
+ */
+int dit_attn_wait_selftest(long long limit_ns, dit_stream_t stream);
+
+/*
  * dit_attn_get_status — synchronise `stream`, copy the device status word to
  * *status_host (DIT_OK or DIT_ERR_TIMEOUT) and reset it to DIT_OK.  Returns
  * DIT_OK, or DIT_ERR_CUDA if the synchronisation or copy failed (for example

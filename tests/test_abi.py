@@ -200,6 +200,11 @@ def test_merge_argument_errors(lib):
     assert call(lse=0x6001) == dit.DIT_ERR_MISALIGNED
 
 
+def test_wait_selftest_limit_range(lib):
+    assert lib.dit_attn_wait_selftest(999, None) == dit.DIT_ERR_INVALID_ARG
+    assert lib.dit_attn_wait_selftest(2 * 10 ** 9, None) == dit.DIT_ERR_INVALID_ARG
+
+
 def test_get_status_rejects_null(lib):
     assert lib.dit_attn_get_status(None, None) == dit.DIT_ERR_INVALID_ARG
 

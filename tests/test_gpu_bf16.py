@@ -11,6 +11,8 @@ Bars: max-abs <= 2e-2 and mean-abs <= 2e-3 on every checked output element,
   operand rounding alone moves O by up to ~8 against the exact oracle, and
   rounding O itself to bf16 costs ~0.12; both are reported, not gated.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -244,3 +246,22 @@ def test_ulysses_single_rank_runs_the_library_kernel():
     b, lb = dit.forward(qd, kd, vd, c, s, n_txt=w.n_txt)
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_bounded_wait_times_out_reports_and_leaves_the_context_usable():
+    """A device wait that nothing completes gives up after its limit, the
+    status word reports DIT_ERR_TIMEOUT once, and the next forward runs
+    normally."""
+    lib = dit.load_library()
+    stream = torch.cuda.current_stream()
+    assert dit.dit_attn_get_status() == dit.DIT_OK
+    assert lib.dit_attn_wait_selftest(10 ** 7, ctypes.c_void_p(stream.cuda_stream)) == dit.DIT_OK   # 10 ms
+    assert dit.dit_attn_get_status() == dit.DIT_ERR_TIMEOUT
+    assert dit.dit_attn_get_status() == dit.DIT_OK                  # read once, then cleared
+    w = W.WORKLOADS["tiny_256"]
+    inputs = device_inputs(w)
+    q, k, v = inputs[:3]
+    rows = W.sample_rows(w)
+    out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
+    O_op, L_op = oracle_rows(w, q, k, v, rows, operands="bf16")
+    check(out32, lse32, rows, O_op, L_op, "after a timed-out wait")
