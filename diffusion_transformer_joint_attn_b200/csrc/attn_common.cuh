@@ -103,9 +103,12 @@ struct SoftmaxIo {
 // (the FP8 operands' scales): within a 128-key tile the first and second 64
 // keys have their own factor, folded into the exponent's fused multiply-add.
 // The running maximum is kept lazily: P = 2^((s - m_used) c) with m_used
-// raised only when a tile's maximum exceeds it by more than 8 (log2 units),
-// so P stays in [0, 256]; the raise rescales O in tensor memory and is
-// warp-uniform because tcgen05 loads / stores are warp-collective.
+// raised only when a tile's maximum exceeds it by more than 15 (log2 units),
+// so P stays in [0, 2^15], below the fp16 maximum (fp16 rounding is relative,
+// so the size of P costs no precision, and a higher threshold means fewer
+// rescales of O on rows whose maximum keeps growing); the raise rescales O in
+// tensor memory and is warp-uniform because tcgen05 loads / stores are
+// warp-collective.
 template <bool kScaled, bool kSparse = false>
 __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem, const Pair& pr, int warp, int lane,
                                              const WaitCtx& wc) {
@@ -117,7 +120,7 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
   const uint32_t tO = tmem + lane_base + 256 + t * 128;
   const uint32_t p_ready_even = cl(&io.p_ready[t], 0);
   const float c = io.scale_log2;
-  const float rescale_gap = 8.0f / c;
+  const float rescale_gap = 15.0f / c;
   const int last_valid = io.N - (io.n_kv - 1) * kTile;
   const int n = pr.row0[t] + row;
   float qs = 1.0f;
