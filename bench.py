@@ -297,6 +297,48 @@ def time_sparse(args, w, lib, q, k_rot, v_f16, cos, sin, out, lse, stream, dev, 
                          "traffic": None, "kernel": "attn_fwd_bf16_kernel (block-sparse)", "peak_source": src}}
 
 
+def time_flushed(args, w, launch, stream, dev, l2_flush_bytes=256 << 20):
+    """Mean duration of `launch` with a 256 MB device write between calls,
+    so that each call starts with a cold L2 (the unflushed number relies on
+    the inputs being larger than L2 instead)."""
+    import torch
+    scratch = torch.empty(l2_flush_bytes, dtype=torch.uint8, device=dev)
+    steps = max(1, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    launch()
+    for a, b in ev:
+        scratch.fill_(1)
+        a.record(stream)
+        launch()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
+def time_sdpa_context(args, w, q, k, v, stream, dev):
+    """Context only: torch's scaled_dot_product_attention (the backend torch
+    picks on this GPU) on the same bf16 [B, H, N, D] shape without rotary
+    embedding and without the LSE.  A library call, not this path."""
+    import torch
+    import torch.nn.functional as F
+    try:
+        for _ in range(2):
+            F.scaled_dot_product_attention(q, k, v)
+        torch.cuda.synchronize(dev)
+        steps = max(1, min(args.steps, 10))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            F.scaled_dot_product_attention(q, k, v)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / steps
+        return {"value": w.flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms": ms,
+                "what": "torch.nn.functional.scaled_dot_product_attention, bf16, no rotary, no LSE (library)"}
+    except Exception as e:       # context only: a missing backend is reported, not fatal
+        return {"unavailable": str(e)[:200]}
+
+
 def time_merge(args, w, lib, out, lse, stream, dev):
     """dit_attn_merge of R = 2 bf16 partial results of the workload's shape
     (a 2-way context-parallel split); memory-bound, reported in GB/s of the
@@ -414,6 +456,13 @@ def run_native(args):
     merge = time_merge(args, w, lib, out, lse, stream, dev)
     sparse = time_sparse(args, w, lib, q, k_rot, v_f16, cos, sin, out, lse, stream, dev, kern_ms)
 
+    def attn_launch():
+        assert lib.dit_attn_forward(q.data_ptr(), k_rot.data_ptr(), v_f16.data_ptr(), cos.data_ptr(), sin.data_ptr(),
+                                    out.data_ptr(), lse.data_ptr(), w.B, w.H, w.n_txt, w.n_img, w.D, flags,
+                                    s_ptr) == 0
+    kern_ms_flushed = time_flushed(args, w, attn_launch, stream, dev)
+    sdpa = time_sdpa_context(args, w, q, k, v, stream, dev)
+
     # end to end through the public C ABI with host buffers: pinned q, k, v
     # and positions in, O and LSE out; dit_attn_forward_host moves chunks of
     # E2E_CHUNK_HEADS heads through a device workspace, overlapping its copies
@@ -477,7 +526,8 @@ def run_native(args):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "attn_fwd_bf16_kernel", "peak_source": peak_src,
-                         "kernel_ms": kern_ms},
+                         "kernel_ms": kern_ms, "kernel_ms_l2_flushed": kern_ms_flushed,
+                         "achieved_l2_flushed": w.flops / (kern_ms_flushed * 1e-3) / 1e12},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / e2e_steps,
                     "api": "dit_attn_forward_host, %d heads per chunk, pinned host buffers" % E2E_CHUNK_HEADS},
@@ -485,6 +535,7 @@ def run_native(args):
             "fp8": fp8,
             "merge": merge,
             "sparse": sparse,
+            "context_library_sdpa": sdpa,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
