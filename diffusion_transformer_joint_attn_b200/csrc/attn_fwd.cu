@@ -16,12 +16,21 @@
 //                 4-slot rings
 //   warp 1        MMA issuer (even CTA only): S_t = Q_t K_j^T (bf16),
 //                 O_t += P_t V_j (fp16, P from tensor memory)
-//   warps 2-15    rotary embedding of the CTA's two Q tiles, once
+//   warps 2-11    rotary embedding of the CTA's two Q tiles, once (and
+//   (2-15)        warps 12-15 where they exist)
 //   warps 2-3,    in-loop operand work when K / V were not prepared by
 //   12-15         dit_attn_prepare_kv: rotation of the K_j half and the exact
 //                 bf16 -> fp16 conversion of the V_j half, in shared memory
 //   warps 4-7     softmax of slot 0 (one thread per query row)
 //   warps 8-11    softmax of slot 1
+//
+// On prepared operands the CTA has 12 warps: 65536 / 384 threads leaves 168
+// registers per thread, enough for a softmax thread's 128 logits, so no
+// register reallocation is needed.  With in-loop operand work it has 16
+// warps, and setmaxnreg moves registers from warpgroups 0 and 3 to the
+// softmax warpgroups.  Only that instance contains setmaxnreg: measured on
+// the B200, a kernel that contains it (even unexecuted) issues the pair MMAs
+// of this loop at 74-86 % of the rate of the same kernel without it.
 //
 // Tensor memory per CTA (512 columns): S_0 | S_1 | O_0 | O_1, 128 lanes x 128
 // fp32 columns each; P_t (fp16) overwrites the first 64 columns of S_t.
@@ -46,14 +55,16 @@ constexpr int kQBoxBytes = kTile * 64 * 2;         // 16 KB: 128 rows x 64 chann
 constexpr int kKHalfBytes = 64 * kHeadDim * 2;     // 16 KB: 64 keys x 128 channels
 constexpr int kKBoxBytes = 64 * 64 * 2;            // 8 KB: 64 keys x 64 channels
 constexpr int kVHalfBytes = kTile * 64 * 2;        // 16 KB: 128 keys x 64 channels
-constexpr int kThreads = 512;
+// Threads per CTA: 12 warps on prepared operands, 16 with in-loop operand work.
+template <bool kPrepared>
+constexpr int kThreadsOf = kPrepared ? 384 : 512;
 constexpr int kProWarps = 6;                       // in-loop operand warps per CTA
 constexpr int kProThreads = kProWarps * 32;
-constexpr int kQRotThreads = 14 * 32;              // warps 2-15 rotate Q
 constexpr int kBarQRot = 1;                        // named barrier of the Q rotation
 constexpr int kMaxKvTiles = 4096;                  // block-sparse launches: N <= 4096 x 128 keys
-// Register split of the 4 x 128 x 128 launch registers between warpgroups:
-// producer / MMA warpgroup, the two softmax warpgroups, the operand warpgroup.
+// Register split of the 4 x 128 x 128 launch registers of the 16-warp CTA
+// between warpgroups: producer / MMA warpgroup, the two softmax warpgroups,
+// the operand warpgroup.
 constexpr uint32_t kIssueRegs = 80;
 constexpr uint32_t kSoftmaxRegs = 184;
 constexpr uint32_t kOperandRegs = 64;
@@ -330,19 +341,20 @@ __device__ __forceinline__ void mma_role(Smem& sm, const Params& p, uint32_t tme
 }
 
 // ---------------------------------------------------------------- operand work
-// Rotary embedding of the CTA's two Q tiles by warps 2-15, then one arrive on
-// the even CTA's q_ready.  kBatch: loads in flight per thread.
-template <int kBatch>
+// Rotary embedding of the CTA's two Q tiles by warps 2 .. (kRotThreads / 32
+// + 1), then one arrive on the even CTA's q_ready.  kBatch: loads in flight
+// per thread.
+template <int kBatch, int kRotThreads>
 __device__ __forceinline__ void rotate_q(Smem& sm, const Params& p, const Pair& pr, int warp, int lane,
                                          const WaitCtx& wc) {
-  const int qt = (warp - 2) * 32 + lane;      // 0..447
+  const int qt = (warp - 2) * 32 + lane;      // 0 .. kRotThreads - 1
   const bool ok = warp_wait(&sm.q_full, 0, wc);
   if (ok && p.cos != nullptr) {
-    rotate_chunks<kQTileBytes / 16, kQRotThreads, kBatch, false>(sm.q[0], pr.row0[0], p, qt);
-    rotate_chunks<kQTileBytes / 16, kQRotThreads, kBatch, false>(sm.q[1], pr.row0[1], p, qt);
+    rotate_chunks<kQTileBytes / 16, kRotThreads, kBatch, false>(sm.q[0], pr.row0[0], p, qt);
+    rotate_chunks<kQTileBytes / 16, kRotThreads, kBatch, false>(sm.q[1], pr.row0[1], p, qt);
   }
   fence_proxy_async_smem();
-  named_bar_sync(kBarQRot, kQRotThreads);
+  named_bar_sync(kBarQRot, kRotThreads);
   if (ok && qt == 0) mbar_arrive_cluster(cl(&sm.q_ready, 0));
 }
 
@@ -372,7 +384,7 @@ __device__ __forceinline__ void kv_prologue_role(Smem& sm, const Params& p, cons
 }
 
 template <bool kPrepared, bool kSparse>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsOf<kPrepared>, 1)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -418,25 +430,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wc{&sm.abort, p.status, cl(&sm.abort, pr.peer)};
 
+  constexpr int kRotThreads = kThreadsOf<kPrepared> - 64;   // warps 2 and up
   const int wg = warp >> 2;
   if (wg == 1 || wg == 2) {
-    regs_increase<kSoftmaxRegs>();
-    rotate_q<4>(sm, p, pr, warp, lane, wc);
+    if constexpr (!kPrepared) regs_increase<kSoftmaxRegs>();
+    rotate_q<4, kRotThreads>(sm, p, pr, warp, lane, wc);
     attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.n_kv, p.out_f32, p.scale_log2,
                        nullptr, nullptr, 0, kv_list(sm), kv_steps<kSparse>(sm, p)};
     attn::softmax_slot<false, kSparse>(io, tmem, pr, warp, lane, wc);
   } else {
-    if (wg == 0)
-      regs_decrease<kIssueRegs>();
-    else
-      regs_decrease<kOperandRegs>();
+    if constexpr (!kPrepared) {
+      if (wg == 0)
+        regs_decrease<kIssueRegs>();
+      else
+        regs_decrease<kOperandRegs>();
+    }
     if (warp == 0) {
       if (lane == 0) producer_role<kPrepared, kSparse>(sm, p, &tm_q, &tm_k, &tm_v, pr, wc);
     } else if (warp == 1) {
       if (lane == 0 && pr.rank == 0) mma_role<kPrepared, kSparse>(sm, p, tmem, wc);
     } else {
-      rotate_q<2>(sm, p, pr, warp, lane, wc);
-      if (!kPrepared) kv_prologue_role<kSparse>(sm, p, pr, warp, lane, wc);
+      rotate_q<2, kRotThreads>(sm, p, pr, warp, lane, wc);
+      if constexpr (!kPrepared) kv_prologue_role<kSparse>(sm, p, pr, warp, lane, wc);
     }
   }
 
@@ -478,7 +493,7 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kThreadsOf<kPrepared>, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
