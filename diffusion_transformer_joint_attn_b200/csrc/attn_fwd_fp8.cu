@@ -8,12 +8,14 @@
 //     a kind::f8f6f4 pair MMA on the codes; the softmax multiplies each half
 //     of a key tile by q_scale(row block) * k_scale(key block), folded into
 //     its exponent's fused multiply-add.
-//   * V arrives as E4M3 codes + scales; warps 2-3 and 12-15 turn each V half
-//     tile into fp16 values code * scale (fp32 product, rounded once) in the
+//   * V arrives as E4M3 codes + scales; warps 2-3 turn each V half tile into
+//     fp16 values code * scale (fp32 product, rounded once) in the
 //     128B-swizzled layout the P V MMA reads, so P V keeps fp16 precision.
 //
-// Roles, by warp:   0 TMA producer | 1 MMA issuer (even CTA) | 2-3, 12-15 V
-// dequantisation | 4-7, 8-11 softmax of slot 0 / 1.
+// Roles, by warp:   0 TMA producer | 1 MMA issuer (even CTA) | 2-3 V
+// dequantisation | 4-7, 8-11 softmax of slot 0 / 1.  Twelve warps leave 168
+// registers per thread (65536 / 384), enough for a softmax row without
+// setmaxnreg, whose mere presence in a kernel slows its pair-MMA issue.
 #include "attn_common.cuh"
 #include "launch.h"
 
@@ -32,13 +34,9 @@ constexpr int kQ8Bytes = kTile * kHeadDim;         // 16 KB: 128 rows x 128 code
 constexpr int kK8HalfBytes = 64 * kHeadDim;        // 8 KB: 64 keys x 128 codes
 constexpr int kV8HalfBytes = kTile * 64;           // 8 KB: 128 keys x 64 codes, unswizzled
 constexpr int kVHalfBytes = kTile * 64 * 2;        // 16 KB: 128 keys x 64 fp16, 128B swizzle
-constexpr int kThreads = 512;
-constexpr int kCvtWarps = 6;
+constexpr int kThreads = 384;
+constexpr int kCvtWarps = 2;                       // warps 2-3
 constexpr int kCvtThreads = kCvtWarps * 32;
-constexpr uint32_t kIssueRegs = 80;
-constexpr uint32_t kSoftmaxRegs = 184;
-constexpr uint32_t kOperandRegs = 64;
-static_assert(kIssueRegs + 2 * kSoftmaxRegs + kOperandRegs == 4 * 128, "register split must use the launch budget");
 
 struct __align__(1024) Smem {
   uint8_t q[2][kQ8Bytes];
@@ -169,11 +167,11 @@ __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t two) {
   return __half22float2(*reinterpret_cast<__half2*>(&h));
 }
 
-// Warps 2-3, 12-15: V_j codes -> fp16 values code * scale in the swizzled
-// operand layout (row = key, 8-channel chunk c at chunk c ^ (key & 7)).
+// Warps 2-3: V_j codes -> fp16 values code * scale in the swizzled operand
+// layout (row = key, 8-channel chunk c at chunk c ^ (key & 7)).
 __device__ __forceinline__ void dequant_v_role(Smem& sm, const Params& p, const Pair& pr, int warp, int lane,
                                                const WaitCtx& wc) {
-  const int pt = (warp < 4 ? (warp - 2) * 32 : 64 + (warp - 12) * 32) + lane;
+  const int pt = (warp - 2) * 32 + lane;
   const float* vscale = p.v_scale + static_cast<size_t>(pr.bh) * p.n_blocks;
   for (int j = 0; j < p.n_kv; ++j) {
     const int s = j % kStages;
@@ -249,16 +247,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int wg = warp >> 2;
   if (wg == 1 || wg == 2) {
-    regs_increase<kSoftmaxRegs>();
     const size_t base = static_cast<size_t>(pr.bh) * p.n_blocks;
     attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.n_kv, p.out_f32, p.scale_log2,
                        p.q_scale + base, p.k_scale + base, p.n_blocks, nullptr, p.n_kv};
     attn::softmax_slot<true>(io, tmem, pr, warp, lane, wc);
   } else {
-    if (wg == 0)
-      regs_decrease<kIssueRegs>();
-    else
-      regs_decrease<kOperandRegs>();
     if (warp == 0) {
       if (lane == 0) producer_role(sm, p, &tm_q, &tm_k, &tm_v, pr, wc);
     } else if (warp == 1) {
