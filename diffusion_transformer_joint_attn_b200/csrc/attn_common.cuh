@@ -11,7 +11,11 @@ namespace attn {
 
 constexpr int kTile = 128;                         // query rows per tile = keys per K/V tile
 constexpr int kHeadDim = 128;
-constexpr int kPolyEvery = 4;                      // every kPolyEvery-th exponent pair on the FMA pipe (0: none)
+// Every kPolyEvery-th exponent pair runs on the FMA pipe (0: none), per
+// kernel: measured best at one pair in four for the BF16 kernel and one in
+// three for the FP8 kernel (whose shorter Q K^T leaves the softmax less time).
+template <bool kScaled>
+constexpr int kPolyEvery = kScaled ? 3 : 4;
 
 struct Pair {
   uint32_t rank;      // 0: even (MMA-issuing) CTA, 1: odd CTA
@@ -56,14 +60,14 @@ __device__ __forceinline__ float max64(const float* f) {
 
 // P for 2 kPairs consecutive logits of the row: 2^(s c - m c) rounded to
 // fp16, packed in pairs into pk[kPairs]; adds the rounded values to sum[4].
-template <int kPairs>
+template <int kPairs, int kPoly>
 __device__ __forceinline__ void exp_pairs(const float* f, float c, float neg, uint32_t* pk, float* sum) {
   const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
 #pragma unroll
   for (int i = 0; i < kPairs; ++i) {
     const float2 x = __ffma2_rn(make_float2(f[2 * i], f[2 * i + 1]), c2, n2);
     float e0, e1;
-    if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
+    if (kPoly > 0 && i % kPoly == kPoly - 1) {
       exp2_pair_poly(x.x, x.y, e0, e1);
     } else {
       e0 = ex2_approx(x.x);
@@ -75,8 +79,9 @@ __device__ __forceinline__ void exp_pairs(const float* f, float c, float neg, ui
     sum[i & 3] = add_f16x2_to_f32(sum[i & 3], pk[i]);
   }
 }
+template <int kPoly>
 __device__ __forceinline__ void exp_half(const float* f, float c, float neg, uint32_t* pk, float* sum) {
-  exp_pairs<32>(f, c, neg, pk, sum);
+  exp_pairs<32, kPoly>(f, c, neg, pk, sum);
 }
 
 // Barriers, outputs and (FP8 only) block scales of one CTA's softmax warps.
@@ -168,9 +173,9 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
     const float neg = -m_used * c;
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
     uint32_t pk[32];
-    exp_half(f, kScaled ? c * sc0 : c, neg, pk, sum);
+    exp_half<kPolyEvery<kScaled>>(f, kScaled ? c * sc0 : c, neg, pk, sum);
     tmem_st32(tS, pk);
-    exp_half(f + 64, kScaled ? c * sc1 : c, neg, pk, sum);
+    exp_half<kPolyEvery<kScaled>>(f + 64, kScaled ? c * sc1 : c, neg, pk, sum);
     tmem_st32(tS + 32, pk);
     l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     if (rescale) {
