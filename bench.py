@@ -155,24 +155,34 @@ def measured_hbm():
     return 6650.0
 
 
-def profile_traffic(kernel_source_sha: str, kernel: str):
+# The translation unit of each profiled kernel; its counters stay valid while
+# that file and the shared headers are unchanged.
+KERNEL_SOURCES = {"attn_fwd_bf16_kernel": "attn_fwd.cu", "attn_fwd_fp8_kernel": "attn_fwd_fp8.cu",
+                  "merge_kernel": "merge.cu"}
+
+
+def profile_traffic(kernel: str):
     """DRAM bytes per launch of `kernel` on the bench workload from the
-    committed ncu summary, or None if none exists for the current source."""
+    committed ncu summary, or None if none was taken of the kernel's current
+    source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("source_sha") != kernel_source_sha or d.get("workload") != WORKLOAD:
+    entry = d.get("kernels", {}).get(kernel, {})
+    if d.get("workload") != WORKLOAD or entry.get("source_sha") != kernel_source_sha(kernel):
         return None
-    return d.get("kernels", {}).get(kernel, {}).get("dram_bytes_per_launch")
+    return entry.get("dram_bytes_per_launch")
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(kernel: str) -> str:
+    """Hash of the kernel's .cu file and every header in csrc/."""
     import hashlib
     csrc = os.path.join(ROOT, "diffusion_transformer_joint_attn_b200", "csrc")
+    names = [KERNEL_SOURCES[kernel]] + sorted(n for n in os.listdir(csrc) if n.endswith((".cuh", ".h")))
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -251,7 +261,7 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
             "gpu_launches": 4 * steps,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "kernel": "attn_fwd_fp8_kernel",
-                         "traffic": profile_traffic(kernel_source_sha(), "attn_fwd_fp8_kernel")
+                         "traffic": profile_traffic("attn_fwd_fp8_kernel")
                          if w.name == WORKLOAD else None,
                          "peak_source": src + " x 4/3 (q k^T at the nominal 2x E4M3 rate, P V at the bf16 rate)",
                          "kernel_ms": kern_ms}}
@@ -378,7 +388,7 @@ def time_merge(args, w, lib, out, lse, stream, dev):
     return {"R": R, "bytes_per_launch": nbytes, "kernel_ms": ms, "launches": steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "kernel": "merge_kernel",
-                         "traffic": profile_traffic(kernel_source_sha(), "merge_kernel") if w.name == WORKLOAD
+                         "traffic": profile_traffic("merge_kernel") if w.name == WORKLOAD
                          else None,
                          "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
 
@@ -509,7 +519,7 @@ def run_native(args):
 
     peak, peak_src = measured_peaks()
     achieved = w.flops / (kern_ms * 1e-3) / 1e12
-    traffic = profile_traffic(kernel_source_sha(), "attn_fwd_bf16_kernel") if w.name == WORKLOAD else None
+    traffic = profile_traffic("attn_fwd_bf16_kernel") if w.name == WORKLOAD else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
