@@ -5,7 +5,10 @@
 // entries (x c - y s with both products exact, one rounding) and rounded to
 // fp32.  The block's scale is amax / 448 in fp32 (1 for an all-zero block);
 // each element becomes the E4M3 code of the fp32 quotient x / scale, rounded
-// to nearest even and saturated to +-448.
+// to nearest even and saturated to +-448.  The quotient comes from one
+// multiplication by the block's reciprocal scale whenever that decides the
+// code (e4m3_of_quotient); the IEEE division runs only for quotients within
+// a few ulps of an E4M3 rounding midpoint.
 #include <cuda_fp8.h>
 
 #include "launch.h"
@@ -24,10 +27,29 @@ __device__ __forceinline__ float rot_f64(float a, float c, float b, float d) {
   return static_cast<float>(fma(static_cast<double>(a), static_cast<double>(c), bd));
 }
 
-__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+// E4M3 codes of lo (low byte) and hi (high byte), nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// E4M3 code of the correctly rounded fp32 quotient x / scale from
+// r = 1 / scale rounded to nearest (scale and r normal); false if undecided.
+// x * r is within 3 fp32 ulps of that quotient: r and the product are each
+// rounded once, with relative error at most 2^-24.  Rounding to E4M3 is
+// monotonic, so when the fp32 values 8 ulps below and above x * r (the lower
+// magnitude clamped at 0) have one code, the quotient has it too.  They
+// differ when the quotient lies within a few ulps of an E4M3 rounding
+// midpoint (or is not finite); the caller then divides.
+__device__ __forceinline__ bool e4m3_of_quotient(float x, float r, uint32_t& code) {
+  const uint32_t u = __float_as_uint(x * r);
+  const uint32_t mag = u & 0x7FFFFFFFu;
+  const float below = __uint_as_float((u & 0x80000000u) | (max(mag, 8u) - 8u));
+  const float above = __uint_as_float(u + 8u);
+  const uint32_t two = e4m3x2(below, above);
+  code = two & 0xFFu;
+  return ((two ^ (two >> 8)) & 0xFFu) == 0u;
 }
 
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
@@ -48,14 +70,20 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
       const long long idx = (static_cast<long long>(bh) * N + n) * 16 + (c & 15);
       const uint4 w = __ldg(x + idx);
       const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      float cs[4] = {}, sn[4] = {};
+      if (tc != nullptr) {
+        // the four pairs of this chunk: table entries n * 64 + (c & 15) * 4 + 0..3
+        const float4 c4 = __ldg(reinterpret_cast<const float4*>(tc) + n * 16 + (c & 15));
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(ts) + n * 16 + (c & 15));
+        cs[0] = c4.x, cs[1] = c4.y, cs[2] = c4.z, cs[3] = c4.w;
+        sn[0] = s4.x, sn[1] = s4.y, sn[2] = s4.z, sn[3] = s4.w;
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float a = __uint_as_float(ww[e] << 16), b = __uint_as_float(ww[e] & 0xFFFF0000u);
         if (tc != nullptr) {
-          const int j = n * 64 + (c & 15) * 4 + e;
-          const float cs = __ldg(tc + j), sn = __ldg(ts + j);
-          v[u][2 * e] = rot_f64(a, cs, b, -sn);
-          v[u][2 * e + 1] = rot_f64(a, sn, b, cs);
+          v[u][2 * e] = rot_f64(a, cs[e], b, -sn[e]);
+          v[u][2 * e + 1] = rot_f64(a, sn[e], b, cs[e]);
         } else {
           v[u][2 * e] = a;
           v[u][2 * e + 1] = b;
@@ -74,21 +102,32 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
   for (int w = 1; w < kThreads / 32; ++w) bmax = fmaxf(bmax, warp_max[w]);
   const float scale = bmax == 0.f ? 1.0f : __fdiv_rn(bmax, 448.0f);
   if (threadIdx.x == 0) scales[blockIdx.x] = scale;
+  // the reciprocal path needs scale and 1 / scale normal: scale in [2^-126, 2^126]
+  const bool via_reciprocal = scale >= 1.17549435e-38f && scale <= 8.50705917e+37f;
+  const float r = __frcp_rn(scale);
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
     const int c = threadIdx.x + u * kThreads;
     const int n = n0 + (c >> 4);
     if (n >= N) continue;
-    uint32_t lo = 0, hi = 0;
+    uint32_t word[2] = {0u, 0u};
+    uint32_t divide = via_reciprocal ? 0u : 0xFFu;   // elements whose quotient needs the division
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t two = e4m3x2(__fdiv_rn(v[u][2 * e], scale), __fdiv_rn(v[u][2 * e + 1], scale));
-      if (e < 2)
-        lo |= two << (16 * e);
-      else
-        hi |= two << (16 * (e - 2));
+    for (int e = 0; e < 8; ++e) {
+      uint32_t code;
+      if (!e4m3_of_quotient(v[u][e], r, code)) divide |= 1u << e;
+      word[e >> 2] |= code << (8 * (e & 3));
     }
-    codes[(static_cast<long long>(bh) * N + n) * 16 + (c & 15)] = make_uint2(lo, hi);
+    if (divide != 0u) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (divide & (1u << e)) {
+          const uint32_t code = e4m3x2(__fdiv_rn(v[u][e], scale), 0.f) & 0xFFu;
+          word[e >> 2] = (word[e >> 2] & ~(0xFFu << (8 * (e & 3)))) | (code << (8 * (e & 3)));
+        }
+      }
+    }
+    codes[(static_cast<long long>(bh) * N + n) * 16 + (c & 15)] = make_uint2(word[0], word[1]);
   }
 }
 

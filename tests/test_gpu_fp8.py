@@ -22,7 +22,7 @@ from oracle import attention as oracle_attention
 from oracle import fp8 as oracle_fp8
 from oracle import rope as oracle_rope
 
-from gpu_cases import BF16_MAX_ABS, BF16_MEAN_ABS, errors, gather_rows, lse_bound
+from gpu_cases import BF16_MAX_ABS, BF16_MEAN_ABS, errors, gather_rows, lse_bound, near_midpoint_blocks
 
 pytestmark = pytest.mark.gpu
 
@@ -122,6 +122,22 @@ def test_quantiser_zero_block_has_scale_one():
     assert scales[0, 0, 0].item() == 1.0
     assert int(codes[..., :64, :].to(torch.int32).sum()) == 0
     check_quantiser(w, q, k, v)
+
+
+def test_quantiser_bitexact_near_e4m3_midpoints():
+    """Quotients x / scale on or within a few fp32 ulps of the midpoints
+    between neighbouring E4M3 values, exact ties included (blocks with
+    power-of-two scales): the codes are those of the correctly rounded fp32
+    quotient, rounded to nearest even, and the scales amax / 448."""
+    x = near_midpoint_blocks()
+    codes_ref, scales_ref = oracle_fp8.quantize(x)
+    assert oracle_fp8.tie_count(x, scales_ref) > 1000      # the ties are there
+    xb = torch.from_numpy(x).to(torch.bfloat16)            # exact: every value is a bf16 value
+    assert torch.equal(xb.float(), torch.from_numpy(x))
+    codes, scales = dit.quantize_fp8(xb.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(scales.cpu().numpy(), scales_ref)
+    assert np.array_equal(codes.cpu().numpy(), codes_ref)
 
 
 # ------------------------------------------------------------------ attention
