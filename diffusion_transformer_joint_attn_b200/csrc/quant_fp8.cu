@@ -52,14 +52,32 @@ __device__ __forceinline__ bool e4m3_of_quotient(float x, float r, uint32_t& cod
   return ((two ^ (two >> 8)) & 0xFFu) == 0u;
 }
 
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
-                                                            const float* __restrict__ ts, uint2* __restrict__ codes,
-                                                            float* __restrict__ scales, int N, int blocks_per_bh) {
+// Element e (0..7) of a chunk held as fp32 values (rotated) or as the raw
+// bf16 words (unrotated: half the registers, so more CTAs stay resident).
+template <bool kRotate>
+struct Chunk;
+template <>
+struct Chunk<true> {
+  float v[8];
+  __device__ __forceinline__ float get(int e) const { return v[e]; }
+};
+template <>
+struct Chunk<false> {
+  uint32_t w[4];
+  __device__ __forceinline__ float get(int e) const {
+    return (e & 1) ? __uint_as_float(w[e >> 1] & 0xFFFF0000u) : __uint_as_float(w[e >> 1] << 16);
+  }
+};
+
+template <bool kRotate>
+__device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, const float* __restrict__ tc,
+                                               const float* __restrict__ ts, uint2* __restrict__ codes,
+                                               float* __restrict__ scales, int N, int blocks_per_bh) {
   __shared__ float warp_max[kThreads / 32];
   const int bh = blockIdx.x / blocks_per_bh;
   const int blk = blockIdx.x % blocks_per_bh;
   const int n0 = blk * kBlockTokens;
-  float v[kPerThread][8];
+  Chunk<kRotate> ch[kPerThread];
   float amax = 0.f;
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
@@ -69,28 +87,23 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
     if (n < N) {
       const long long idx = (static_cast<long long>(bh) * N + n) * 16 + (c & 15);
       const uint4 w = __ldg(x + idx);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-      float cs[4] = {}, sn[4] = {};
-      if (tc != nullptr) {
+      if constexpr (kRotate) {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
         // the four pairs of this chunk: table entries n * 64 + (c & 15) * 4 + 0..3
         const float4 c4 = __ldg(reinterpret_cast<const float4*>(tc) + n * 16 + (c & 15));
         const float4 s4 = __ldg(reinterpret_cast<const float4*>(ts) + n * 16 + (c & 15));
-        cs[0] = c4.x, cs[1] = c4.y, cs[2] = c4.z, cs[3] = c4.w;
-        sn[0] = s4.x, sn[1] = s4.y, sn[2] = s4.z, sn[3] = s4.w;
-      }
+        const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a = __uint_as_float(ww[e] << 16), b = __uint_as_float(ww[e] & 0xFFFF0000u);
-        if (tc != nullptr) {
-          v[u][2 * e] = rot_f64(a, cs[e], b, -sn[e]);
-          v[u][2 * e + 1] = rot_f64(a, sn[e], b, cs[e]);
-        } else {
-          v[u][2 * e] = a;
-          v[u][2 * e + 1] = b;
+        for (int e = 0; e < 4; ++e) {
+          const float a = __uint_as_float(ww[e] << 16), b = __uint_as_float(ww[e] & 0xFFFF0000u);
+          ch[u].v[2 * e] = rot_f64(a, cs[e], b, -sn[e]);
+          ch[u].v[2 * e + 1] = rot_f64(a, sn[e], b, cs[e]);
         }
+      } else {
+        ch[u].w[0] = w.x, ch[u].w[1] = w.y, ch[u].w[2] = w.z, ch[u].w[3] = w.w;
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(ch[u].get(e)));
     }
   }
 #pragma unroll
@@ -115,14 +128,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       uint32_t code;
-      if (!e4m3_of_quotient(v[u][e], r, code)) divide |= 1u << e;
+      if (!e4m3_of_quotient(ch[u].get(e), r, code)) divide |= 1u << e;
       word[e >> 2] |= code << (8 * (e & 3));
     }
     if (divide != 0u) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         if (divide & (1u << e)) {
-          const uint32_t code = e4m3x2(__fdiv_rn(v[u][e], scale), 0.f) & 0xFFu;
+          const uint32_t code = e4m3x2(__fdiv_rn(ch[u].get(e), scale), 0.f) & 0xFFu;
           word[e >> 2] = (word[e >> 2] & ~(0xFFu << (8 * (e & 3)))) | (code << (8 * (e & 3)));
         }
       }
@@ -131,14 +144,30 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
   }
 }
 
+// q, k (rotated): 64 registers, 4 CTAs per SM.  v: the raw words take fewer
+// registers, and 5 CTAs per SM keep more loads in flight.
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
+                                                            const float* __restrict__ ts, uint2* __restrict__ codes,
+                                                            float* __restrict__ scales, int N, int blocks_per_bh) {
+  quantize_block<true>(x, tc, ts, codes, scales, N, blocks_per_bh);
+}
+__global__ void __launch_bounds__(kThreads, 5)
+    quantize_unrotated_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes, float* __restrict__ scales, int N,
+                              int blocks_per_bh) {
+  quantize_block<false>(x, nullptr, nullptr, codes, scales, N, blocks_per_bh);
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_fp8(const QuantFp8Args& a, cudaStream_t s) {
   const int blocks_per_bh = (a.N + kBlockTokens - 1) / kBlockTokens;
   const long long grid = static_cast<long long>(a.B) * a.H * blocks_per_bh;
-  quantize_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(static_cast<const uint4*>(a.x), a.cos, a.sin,
-                                                                   static_cast<uint2*>(a.codes), a.scale, a.N,
-                                                                   blocks_per_bh);
+  if (a.cos != nullptr)
+    quantize_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+        static_cast<const uint4*>(a.x), a.cos, a.sin, static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh);
+  else
+    quantize_unrotated_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+        static_cast<const uint4*>(a.x), static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh);
   return cudaGetLastError();
 }
 
