@@ -146,21 +146,40 @@ int dit_attn_forward(const void* q, const void* k, const void* v, const float* r
 
 size_t dit_attn_forward_host_workspace(int B, int H, int N, int D, int dtype, int chunk_heads) {
   if (B < 1 || H < 1 || N < 1 || chunk_heads < 1 || D != 128) return 0;
+  if (static_cast<long long>(B) * H > 0x7FFFFFFF) return 0;
   if ((dtype & ~DIT_OUT_F32) != DIT_BF16) return 0;
   return dit::host_forward_workspace_bytes(B * H, N, chunk_heads, (dtype & DIT_OUT_F32) != 0);
 }
 
-int dit_attn_forward_host(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
-                          void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
-                          void* workspace, size_t workspace_bytes, int chunk_heads, dit_stream_t stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || workspace == nullptr)
-    return DIT_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// The argument checks of the host-buffer entries that need no workspace and
+// no CUDA call.
+int host_forward_args(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                      const void* out, int B, int H, int N_txt, int N_img, int D, int dtype, int chunk_heads) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N_txt < 0 || N_img < 0 || chunk_heads < 1) return DIT_ERR_INVALID_ARG;
   const long long N = static_cast<long long>(N_txt) + N_img;
   if (N < 1 || N > 0x7FFFFFFF || static_cast<long long>(B) * H > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
   if (D != 128) return DIT_ERR_UNSUPPORTED;
   if ((dtype & ~DIT_OUT_F32) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+  return DIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dit_attn_forward_host(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                          void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
+                          void* workspace, size_t workspace_bytes, int chunk_heads, dit_stream_t stream) {
+  const int rc = host_forward_args(q, k, v, rope_cos, rope_sin, out, B, H, N_txt, N_img, D, dtype, chunk_heads);
+  if (rc != DIT_OK) return rc;
+  if (workspace == nullptr) return DIT_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img;
   const bool out_f32 = (dtype & DIT_OUT_F32) != 0;
   if (workspace_bytes < dit::host_forward_workspace_bytes(B * H, static_cast<int>(N), chunk_heads, out_f32))
     return DIT_ERR_INVALID_ARG;
@@ -174,14 +193,15 @@ int dit_attn_forward_host(const void* q, const void* k, const void* v, const flo
 int dit_attn_forward_host_static(const void* q, const void* k, const void* v, const float* rope_cos,
                                  const float* rope_sin, void* out, float* lse, int B, int H, int N_txt, int N_img,
                                  int D, int dtype, int chunk_heads, dit_stream_t stream) {
+  // argument errors and an oversize problem are reported before any CUDA call
+  int rc = host_forward_args(q, k, v, rope_cos, rope_sin, out, B, H, N_txt, N_img, D, dtype, chunk_heads);
+  if (rc != DIT_OK) return rc;
   const long long N = static_cast<long long>(N_txt) + N_img;
-  if (B >= 1 && H >= 1 && N >= 1 && N <= 0x7FFFFFFF && chunk_heads >= 1 && D == 128 &&
-      (dtype & ~DIT_OUT_F32) == DIT_BF16 &&
-      dit::host_forward_workspace_bytes(B * H, static_cast<int>(N), chunk_heads, (dtype & DIT_OUT_F32) != 0) >
-          DIT_STATIC_WORKSPACE_BYTES)
+  if (dit::host_forward_workspace_bytes(B * H, static_cast<int>(N), chunk_heads, (dtype & DIT_OUT_F32) != 0) >
+      DIT_STATIC_WORKSPACE_BYTES)
     return DIT_ERR_WORKSPACE;
   void* ws = nullptr;
-  const int rc = cuda_status(dit::static_workspace(&ws));
+  rc = cuda_status(dit::static_workspace(&ws));
   if (rc != DIT_OK) return rc;
   return dit_attn_forward_host(q, k, v, rope_cos, rope_sin, out, lse, B, H, N_txt, N_img, D, dtype, ws,
                                DIT_STATIC_WORKSPACE_BYTES, chunk_heads, stream);

@@ -117,6 +117,28 @@ def test_static_workspace_entry_rejects_oversize_without_a_gpu(lib):
     assert dit.dit_attn_status_string(rc) == "problem needs more workspace than the static workspace holds"
 
 
+def test_static_workspace_entry_argument_errors_before_any_cuda_call(lib):
+    f = lib.dit_attn_forward_host_static
+
+    def call(q=0x1000, B=1, H=2, nt=16, ni=48, D=128, dtype=0, chunk=1, cos=None, sin=None):
+        return f(q, 0x2000, 0x3000, cos, sin, 0x4000, None, B, H, nt, ni, D, dtype, chunk, None)
+    assert call(q=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(cos=0x5000) == dit.DIT_ERR_INVALID_ARG                    # sin missing
+    assert call(B=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(nt=0, ni=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(chunk=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(B=65536, H=65536) == dit.DIT_ERR_INVALID_ARG             # B * H beyond int
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=dit.DIT_V_F16) == dit.DIT_ERR_UNSUPPORTED
+
+
+def test_host_entries_reject_head_counts_beyond_int(lib):
+    assert lib.dit_attn_forward_host_workspace(65536, 65536, 16, 128, 0, 4) == 0
+    rc = lib.dit_attn_forward_host(0x1000, 0x2000, 0x3000, None, None, 0x4000, None, 65536, 65536, 0, 16, 128, 0,
+                                   0x8000, 1 << 40, 4, None)
+    assert rc == dit.DIT_ERR_INVALID_ARG
+
+
 def test_rope_table_argument_errors(lib):
     ax = (ctypes.c_int32 * 3)(16, 56, 56)
     bad = (ctypes.c_int32 * 3)(16, 55, 57)
