@@ -146,11 +146,13 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
  *
  * Precision: each rotated component of q and k is the bf16 nearest to its
  * exact value for the fp32 table entries; q~ k~^T accumulates in fp32; the
- * softmax runs in fp32; P (in [0, 256]) and v are fp16 tensor-core operands
+ * softmax runs in fp32; P (in [0, 2^15]) and v are fp16 tensor-core operands
  * (v must satisfy |v| <= 65504; the bf16 -> fp16 conversion of v is exact for
  * |v| >= 2^-14), P v accumulates in fp32.
- * All pointers 16-byte aligned except lse (4-byte).  Graph-capturable: one
- * kernel launch, no host synchronisation, no allocation.
+ * All pointers 16-byte aligned except lse (4-byte).  One kernel launch, no
+ * host synchronisation, no allocation.  The first call on a device also sets
+ * the kernel's shared-memory limit and looks up the status word's address;
+ * make it outside any stream capture (capture of later calls is not tested).
  */
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                      void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
