@@ -22,8 +22,10 @@
  *   - Layout: q, k, v, out are [B][H][N][D] row-major, N = N_txt + N_img
  *     tokens in sequence order [text | image(s)]; lse is [B][H][N].
  *   - Ownership: the caller allocates and owns every buffer.  The library
- *     allocates no device memory per call; it keeps one static device status
- *     word.  Inputs are only read; outputs are fully overwritten.
+ *     allocates no device memory per call; its device image holds one status
+ *     word and the DIT_STATIC_WORKSPACE_BYTES array of
+ *     dit_attn_forward_host_static.  Inputs are only read; outputs are fully
+ *     overwritten.
  *   - Streams: every call is asynchronous on `stream` (a cudaStream_t, NULL =
  *     legacy default stream) and does not synchronise the host, except
  *     dit_attn_get_status.
