@@ -62,6 +62,22 @@ def _require(cond: bool, msg: str) -> None:
         raise ValueError(msg)
 
 
+def _on_current_device(*tensors) -> None:
+    """The library launches on the current CUDA device and hands it the
+    tensors' addresses, so every CUDA tensor of a call (None entries are
+    skipped) must live on that one device; anything else is refused here
+    instead of reaching a kernel as another device's address."""
+    devs = {t.device for t in tensors if t is not None and t.is_cuda}
+    _require(len(devs) <= 1, "the CUDA tensors of one call must be on one device, not %s" %
+             ", ".join(sorted(str(d) for d in devs)))
+    if devs:
+        import torch
+        dev = devs.pop()
+        cur = torch.cuda.current_device()
+        _require(dev.index == cur, "the tensors are on %s but the current device is cuda:%d "
+                 "(torch.cuda.set_device selects it)" % (dev, cur))
+
+
 def dit_rope_table_build(pos, axes: Sequence[int], theta: float, rope_cos, rope_sin, stream=None) -> None:
     """Fill rope_cos / rope_sin (CUDA fp32 [N, 64]) from positions pos (CUDA int32 [N, 3])."""
     import torch
@@ -71,6 +87,7 @@ def dit_rope_table_build(pos, axes: Sequence[int], theta: float, rope_cos, rope_
     for t in (rope_cos, rope_sin):
         _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (N, 64),
                  "rope tables must be contiguous CUDA fp32 [N, 64] tensors")
+    _on_current_device(pos, rope_cos, rope_sin)
     ax = (ctypes.c_int32 * 3)(*[int(a) for a in axes])
     _check(load_library().dit_rope_table_build(_ptr(pos), N, 128, ax, float(theta), _ptr(rope_cos),
                                                _ptr(rope_sin), _stream(stream)), "dit_rope_table_build")
@@ -86,6 +103,7 @@ def dit_rope_apply(x, rope_cos, rope_sin, x_rot, stream=None) -> None:
     for t in (rope_cos, rope_sin):
         _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (N, D // 2),
                  "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _on_current_device(x, rope_cos, rope_sin, x_rot)
     _check(load_library().dit_rope_apply(_ptr(x), _ptr(rope_cos), _ptr(rope_sin), _ptr(x_rot), B, H, N, D,
                                          _stream(stream)), "dit_rope_apply")
 
@@ -101,6 +119,7 @@ def dit_attn_prepare_kv(k, v, rope_cos, rope_sin, k_rot, v_f16, stream=None) -> 
     for t in (rope_cos, rope_sin):
         _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (N, D // 2),
                  "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _on_current_device(k, v, rope_cos, rope_sin, k_rot, v_f16)
     _check(load_library().dit_attn_prepare_kv(_ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(k_rot),
                                               _ptr(v_f16), B, H, N, D, _stream(stream)), "dit_attn_prepare_kv")
 
@@ -134,6 +153,7 @@ def _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dty
         for t in (rope_cos, rope_sin):
             _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
                      tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _on_current_device(q, k, v, rope_cos, rope_sin, out, lse)
 
 
 def dit_attn_forward_host_workspace(B: int, H: int, N: int, dtype: int = DIT_BF16, chunk_heads: int = 4) -> int:
@@ -162,6 +182,7 @@ def dit_attn_forward_host(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_i
             _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
                      tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
     _require(workspace.is_cuda and workspace.is_contiguous(), "workspace must be a contiguous CUDA tensor")
+    _on_current_device(rope_cos, rope_sin, workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(load_library().dit_attn_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(out),
                                                 _ptr(lse), B, H, n_txt, n_img, D, dtype, _ptr(workspace), nbytes,
@@ -178,6 +199,7 @@ def dit_attn_forward_sparse(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, n_tx
              and tuple(kv_mask.shape) == (B, H, (N + 511) // 512, (N + 127) // 128),
              "kv_mask must be a contiguous CUDA uint8 [B, H, ceil(N/512), ceil(N/128)] tensor")
     _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dtype)
+    _on_current_device(kv_mask)
     _check(load_library().dit_attn_forward_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin),
                                                   _ptr(kv_mask), _ptr(out), _ptr(lse), B, H, n_txt, n_img, D, dtype,
                                                   _stream(stream)), "dit_attn_forward_sparse")
@@ -196,6 +218,7 @@ def dit_attn_quantize_fp8(x, rope_cos, rope_sin, x_fp8, scale, stream=None) -> N
         for t in (rope_cos, rope_sin):
             _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
                      tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _on_current_device(x, rope_cos, rope_sin, x_fp8, scale)
     _check(load_library().dit_attn_quantize_fp8(_ptr(x), _ptr(rope_cos), _ptr(rope_sin), _ptr(x_fp8), _ptr(scale),
                                                 B, H, N, D, _stream(stream)), "dit_attn_quantize_fp8")
 
@@ -229,6 +252,7 @@ def dit_attn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, n_txt:
     if lse is not None:
         _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, N),
                  "lse must be a contiguous CUDA fp32 [B, H, N] tensor")
+    _on_current_device(q8, k8, v8, q_scale, k_scale, v_scale, out, lse)
     _check(load_library().dit_attn_forward_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale),
                                                _ptr(v_scale), _ptr(out), _ptr(lse), B, H, n_txt, n_img, D, dtype,
                                                _stream(stream)), "dit_attn_forward_fp8")
@@ -252,6 +276,7 @@ def dit_attn_merge(o_parts, lse_parts, out, lse_out=None, dtype: int = DIT_BF16,
     if lse_out is not None:
         _require(lse_out.is_cuda and lse_out.dtype == torch.float32 and lse_out.is_contiguous() and
                  tuple(lse_out.shape) == (B, H, N), "lse_out must be contiguous CUDA fp32 [B, H, N]")
+    _on_current_device(out, lse_out)       # the parts may be a peer GPU's memory, read over NVLink
     optr = (ctypes.c_void_p * R)(*[o.data_ptr() for o in o_parts])
     lptr = (ctypes.c_void_p * R)(*[l.data_ptr() for l in lse_parts])
     _check(load_library().dit_attn_merge(ctypes.cast(optr, ctypes.c_void_p), ctypes.cast(lptr, ctypes.c_void_p), R,

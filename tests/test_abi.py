@@ -231,6 +231,18 @@ def test_get_status_rejects_null(lib):
     assert lib.dit_attn_get_status(None, None) == dit.DIT_ERR_INVALID_ARG
 
 
+def test_binding_refuses_cuda_tensors_on_several_devices():
+    import torch
+
+    class OnDevice:                      # the two attributes the check reads of a CUDA tensor
+        def __init__(self, index):
+            self.is_cuda = True
+            self.device = torch.device("cuda", index)
+    with pytest.raises(ValueError, match="one device"):
+        dit._on_current_device(OnDevice(0), None, OnDevice(1))
+    dit._on_current_device(None, torch.zeros(2))     # no CUDA tensor: nothing to check, no CUDA call
+
+
 def test_binding_marshalling_errors():
     import torch
     q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
