@@ -53,6 +53,23 @@ def _worker(rank, world, port, case, rq):
             lse = x[..., 0]
             lh = ulysses.head_to_seq(lse[:, rank * Hl:(rank + 1) * Hl].unsqueeze(-1)).squeeze(-1)
             result["lse_ok"] = bool(torch.equal(lh, lse[:, :, rank * Ns:(rank + 1) * Ns]))
+        elif case == "errors":
+            # every check fails on every rank before a collective is entered
+            def refused(fn):
+                try:
+                    fn()
+                except ValueError:
+                    return True
+                return False
+            odd_heads = torch.zeros(1, 2 * world + 1, 4, 3)
+            odd_tokens = torch.zeros(1, 1, 2 * world + 1, 3)
+            shard = torch.zeros(1, 2 * world, 4, 3)
+            result["heads"] = refused(lambda: ulysses.seq_to_head(odd_heads))
+            result["tokens"] = refused(lambda: ulysses.head_to_seq(odd_tokens))
+            result["tables"] = refused(lambda: ulysses.ulysses_attention(
+                shard, shard, shard, torch.zeros(4, 64), torch.zeros(4, 64), attn=lambda *a: None))
+            result["shapes"] = refused(lambda: ulysses.ulysses_attention(shard, shard[:, :1], shard))
+            dist.barrier()                        # the ranks are still in step
         else:
             import workloads as W
             from oracle import attention as oracle_attention
@@ -118,6 +135,12 @@ def test_ulysses_attention_matches_full_sequence_oracle(world):
     res = _run(world, "ulysses")
     for rank, r in res.items():
         assert r["max_err"] < 1e-12 and r["lse_err"] < 1e-12, (rank, r)
+
+
+def test_exchange_argument_errors_on_every_rank():
+    res = _run(2, "errors")
+    for rank, r in res.items():
+        assert all(r.values()), (rank, r)
 
 
 def test_cfg_groups_split_the_batch():
