@@ -27,6 +27,7 @@ DIT_OUT_F32 = 0x100
 DIT_K_ROTATED = 0x200
 DIT_V_F16 = 0x400
 DIT_PART_F32 = 0x800
+DIT_QK_SPLIT = 0x1000
 DIT_MERGE_MAX_PARTS = 16
 DIT_SPARSE_MAX_KV_TILES = 4096
 
@@ -124,6 +125,72 @@ def dit_attn_prepare_kv(k, v, rope_cos, rope_sin, k_rot, v_f16, stream=None) -> 
                                               _ptr(v_f16), B, H, N, D, _stream(stream)), "dit_attn_prepare_kv")
 
 
+def dit_attn_prepare_kv_split(k, v, rope_cos, rope_sin, k_split, v_f16, stream=None) -> None:
+    """k_split <- fp16 [2, B, H, N, D] hi / lo split of the rotated k, v_f16 <- fp16 copy of v; the tables may
+    both be None (no rotation)."""
+    import torch
+    _require(k.dim() == 4 and k.shape == v.shape == v_f16.shape, "k, v, v_f16 shapes differ")
+    B, H, N, D = k.shape
+    _require(tuple(k_split.shape) == (2, B, H, N, D), "k_split must be [2, B, H, N, D]")
+    for t in (k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "k, v must be contiguous CUDA bf16")
+    for t in (k_split, v_f16):
+        _require(t.is_cuda and t.dtype == torch.float16 and t.is_contiguous(), "k_split, v_f16 must be CUDA fp16")
+    _check_tables(rope_cos, rope_sin, N, D)
+    _on_current_device(k, v, rope_cos, rope_sin, k_split, v_f16)
+    _check(load_library().dit_attn_prepare_kv_split(_ptr(k), _ptr(v), _ptr(rope_cos), _ptr(rope_sin), _ptr(k_split),
+                                                    _ptr(v_f16), B, H, N, D, _stream(stream)),
+           "dit_attn_prepare_kv_split")
+
+
+def _check_tables(rope_cos, rope_sin, N, D):
+    """Both tables None, or both contiguous CUDA fp32 [N, D/2]."""
+    import torch
+    if rope_cos is not None or rope_sin is not None:
+        for t in (rope_cos, rope_sin):
+            _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+
+
+def dit_attn_forward_kv(q, k, v, q_cos, q_sin, out, lse, dtype: int = DIT_BF16, stream=None) -> None:
+    """out (and lse) <- attention of bf16 q [B, H, N_q, D] to the N_kv keys and values k, v [B, H, N_kv, D]
+    (k: the [2, B, H, N_kv, D] fp16 split operand with DIT_QK_SPLIT); q_cos / q_sin: the queries' table rows."""
+    import torch
+    _require(q.dim() == 4 and v.dim() == 4 and q.shape[:2] == v.shape[:2] and q.shape[3] == v.shape[3],
+             "q [B, H, N_q, D] and v [B, H, N_kv, D] must agree in B, H, D")
+    B, H, N_q, D = q.shape
+    N_kv = v.shape[2]
+    _check_operands(q, k, v, out, lse, dtype, N_kv)
+    _check_tables(q_cos, q_sin, N_q, D)
+    _on_current_device(q, k, v, q_cos, q_sin, out, lse)
+    _check(load_library().dit_attn_forward_kv(_ptr(q), _ptr(k), _ptr(v), _ptr(q_cos), _ptr(q_sin), _ptr(out),
+                                              _ptr(lse), B, H, N_q, N_kv, D, dtype, _stream(stream)),
+           "dit_attn_forward_kv")
+
+
+def _check_operands(q, k, v, out, lse, dtype, N_kv):
+    """dtype / shape checks of q, k, v, out, lse for N_q queries (q.shape[2]) and N_kv keys."""
+    import torch
+    B, H, N_q, D = q.shape
+    _require(q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous(), "q must be contiguous CUDA bf16")
+    if dtype & DIT_QK_SPLIT:
+        _require(tuple(k.shape) == (2, B, H, N_kv, D) and k.is_cuda and k.dtype == torch.float16 and
+                 k.is_contiguous(), "with DIT_QK_SPLIT, k must be the contiguous CUDA fp16 [2, B, H, N_kv, D] "
+                 "operand of dit_attn_prepare_kv_split")
+    else:
+        _require(tuple(k.shape) == (B, H, N_kv, D) and k.is_cuda and k.dtype == torch.bfloat16 and k.is_contiguous(),
+                 "k must be a contiguous CUDA bf16 [B, H, N_kv, D] tensor")
+    v_dtype = torch.float16 if dtype & DIT_V_F16 else torch.bfloat16
+    _require(tuple(v.shape) == (B, H, N_kv, D) and v.is_cuda and v.dtype == v_dtype and v.is_contiguous(),
+             "v must be a contiguous CUDA bf16 (fp16 with DIT_V_F16) [B, H, N_kv, D] tensor")
+    out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
+    _require(out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q.shape,
+             "out must be a contiguous CUDA tensor of q's shape and the requested dtype")
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and
+                 tuple(lse.shape) == (B, H, N_q), "lse must be a contiguous CUDA fp32 [B, H, N_q] tensor")
+
+
 def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: int, dtype: int = DIT_BF16,
                      stream=None) -> None:
     """out (and lse, if not None) <- joint attention of bf16 q, k, v [B, H, N, D] on the GPU."""
@@ -135,24 +202,11 @@ def dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt: int, n_img: i
 
 
 def _check_forward_args(q, k, v, rope_cos, rope_sin, out, lse, n_txt, n_img, dtype):
-    import torch
-    _require(q.dim() == 4 and q.shape == k.shape == v.shape, "q, k, v must share one [B, H, N, D] shape")
+    _require(q.dim() == 4 and v.dim() == 4 and q.shape == v.shape, "q, k, v must share one [B, H, N, D] shape")
     B, H, N, D = q.shape
     _require(N == n_txt + n_img, "N must equal n_txt + n_img")
-    for t in (q, k):
-        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "q, k must be contiguous CUDA bf16")
-    v_dtype = torch.float16 if dtype & DIT_V_F16 else torch.bfloat16
-    _require(v.is_cuda and v.dtype == v_dtype and v.is_contiguous(), "v must be contiguous CUDA bf16 (fp16 with DIT_V_F16)")
-    out_dtype = torch.float32 if dtype & DIT_OUT_F32 else torch.bfloat16
-    _require(out.is_cuda and out.dtype == out_dtype and out.is_contiguous() and out.shape == q.shape,
-             "out must be a contiguous CUDA tensor of q's shape and the requested dtype")
-    if lse is not None:
-        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, N),
-                 "lse must be a contiguous CUDA fp32 [B, H, N] tensor")
-    if rope_cos is not None or rope_sin is not None:
-        for t in (rope_cos, rope_sin):
-            _require(t is not None and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
-                     tuple(t.shape) == (N, D // 2), "rope tables must be contiguous CUDA fp32 [N, D/2]")
+    _check_operands(q, k, v, out, lse, dtype, N)
+    _check_tables(rope_cos, rope_sin, N, D)
     _on_current_device(q, k, v, rope_cos, rope_sin, out, lse)
 
 
@@ -306,15 +360,43 @@ def rope_table(pos, axes=(16, 56, 56), theta: float = 10000.0, stream=None):
     return c, s
 
 
+def _flags(out_f32, k_rotated, v_f16, qk_split):
+    return ((DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0) | (DIT_V_F16 if v_f16 else 0) |
+            (DIT_QK_SPLIT if qk_split else 0))
+
+
 def forward(q, k, v, rope_cos=None, rope_sin=None, n_txt: int = 0, out_f32: bool = False, with_lse: bool = True,
-            k_rotated: bool = False, v_f16: bool = False, stream=None):
-    """Allocate out (and lse) and run dit_attn_forward; returns (out, lse)."""
+            k_rotated: bool = False, v_f16: bool = False, qk_split: bool = False, stream=None):
+    """Allocate out (and lse) and run dit_attn_forward; returns (out, lse).  qk_split: k, v are the
+    operands of prepare_kv_split (v_f16 is implied)."""
     import torch
     B, H, N, D = q.shape
     out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
-    flags = (DIT_OUT_F32 if out_f32 else 0) | (DIT_K_ROTATED if k_rotated else 0) | (DIT_V_F16 if v_f16 else 0)
+    flags = _flags(out_f32, k_rotated, v_f16 or qk_split, qk_split)
     dit_attn_forward(q, k, v, rope_cos, rope_sin, out, lse, n_txt, N - n_txt, DIT_BF16 | flags, stream)
+    return out, lse
+
+
+def prepare_kv_split(k, v, rope_cos=None, rope_sin=None, stream=None):
+    """Allocate and fill (k_split [2, B, H, N, D] fp16, v_f16) for the split form (DIT_QK_SPLIT)."""
+    import torch
+    k_split = torch.empty((2,) + tuple(k.shape), dtype=torch.float16, device=k.device)
+    v_f16 = torch.empty(v.shape, dtype=torch.float16, device=v.device)
+    dit_attn_prepare_kv_split(k, v, rope_cos, rope_sin, k_split, v_f16, stream)
+    return k_split, v_f16
+
+
+def forward_kv(q, k, v, q_cos=None, q_sin=None, out_f32: bool = False, with_lse: bool = True,
+               k_rotated: bool = False, v_f16: bool = False, qk_split: bool = False, stream=None):
+    """Allocate out (and lse) and run dit_attn_forward_kv (queries q against the keys / values k, v);
+    returns (out, lse)."""
+    import torch
+    B, H, N_q, D = q.shape
+    out = torch.empty(q.shape, dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device) if with_lse else None
+    dit_attn_forward_kv(q, k, v, q_cos, q_sin, out, lse, DIT_BF16 | _flags(out_f32, k_rotated, v_f16 or qk_split,
+                                                                        qk_split), stream)
     return out, lse
 
 

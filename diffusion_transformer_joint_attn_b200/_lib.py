@@ -17,7 +17,9 @@ SIGNATURES = {
     "dit_rope_table_build": (_I, [_VP, _I, _I, ctypes.POINTER(ctypes.c_int32), ctypes.c_double, _VP, _VP, _VP]),
     "dit_rope_apply": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_prepare_kv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
+    "dit_attn_prepare_kv_split": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
+    "dit_attn_forward_kv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_host_workspace": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "dit_attn_forward_host": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, ctypes.c_size_t,
                                    _I, _VP]),

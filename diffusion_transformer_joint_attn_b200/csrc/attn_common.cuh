@@ -91,8 +91,9 @@ struct SoftmaxIo {
   uint64_t* o_final;       // [2] local: the last P V product of slot t has completed
   void* out;
   float* lse;
-  int N;
-  int n_kv;
+  int N;                   // query rows per (b, h)
+  int N_kv;                // keys per (b, h)
+  int n_kv;                // key tiles: ceil(N_kv / 128)
   int out_f32;
   float scale_log2;        // log2(e) / sqrt(D)
   const float* q_scale;    // this (b, h)'s per-64-token scales, or nullptr (unscaled logits)
@@ -126,7 +127,7 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
   const uint32_t p_ready_even = cl(&io.p_ready[t], 0);
   const float c = io.scale_log2;
   const float rescale_gap = 15.0f / c;
-  const int last_valid = io.N - (io.n_kv - 1) * kTile;
+  const int last_valid = io.N_kv - (io.n_kv - 1) * kTile;
   const int n = pr.row0[t] + row;
   float qs = 1.0f;
   if (kScaled && n < io.N) qs = __ldg(io.q_scale + n / 64);

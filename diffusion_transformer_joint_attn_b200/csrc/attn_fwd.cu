@@ -94,7 +94,8 @@ struct Params {
   float* lse;
   int* status;
   const uint8_t* kv_mask;   // [B*H][clusters][n_kv] block mask, or nullptr (all key tiles)
-  int N;
+  int N;              // query rows per (b, h)
+  int N_kv;           // keys per (b, h)
   int n_kv;
   int clusters;       // CTA pairs per (b, h): 512 query rows each
   int out_f32;
@@ -176,7 +177,7 @@ __device__ __forceinline__ void rotate_chunks(uint8_t* tile, int n0, const Param
       else
         q_chunk(c < kChunks ? c : 0, off[u], row, col0);
       const int n = n0 + row;
-      live[u] = c < kChunks && n < p.N;
+      live[u] = c < kChunks && n < (kHalfK ? p.N_kv : p.N);
       if (live[u]) {
         const int j0 = n * (kHeadDim / 2) + (col0 >> 1);
         x[u] = *reinterpret_cast<const uint4*>(tile + off[u]);
@@ -435,8 +436,8 @@ __global__ void __launch_bounds__(kThreadsOf<kPrepared>, 1)
   if (wg == 1 || wg == 2) {
     if constexpr (!kPrepared) regs_increase<kSoftmaxRegs>();
     rotate_q<4, kRotThreads>(sm, p, pr, warp, lane, wc);
-    attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.n_kv, p.out_f32, p.scale_log2,
-                       nullptr, nullptr, 0, kv_list(sm), kv_steps<kSparse>(sm, p)};
+    attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.N_kv, p.n_kv, p.out_f32,
+                       p.scale_log2, nullptr, nullptr, 0, kv_list(sm), kv_steps<kSparse>(sm, p)};
     attn::softmax_slot<false, kSparse>(io, tmem, pr, warp, lane, wc);
   } else {
     if constexpr (!kPrepared) {
@@ -510,9 +511,10 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, 
 
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   const int BH = a.B * a.H;
+  const int N_kv = a.N_kv > 0 ? a.N_kv : a.N;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, BH, a.N, false, kTile) || !make_map(&mk, a.k, BH, a.N, false, 64) ||
-      !make_map(&mv, a.v, BH, a.N, a.v_f16, kTile))
+  if (!make_map(&mq, a.q, BH, a.N, false, kTile) || !make_map(&mk, a.k, BH, N_kv, false, 64) ||
+      !make_map(&mv, a.v, BH, N_kv, a.v_f16, kTile))
     return -4;
   Params p;
   p.cos = a.cos;
@@ -523,7 +525,8 @@ int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s) {
   if (p.status == nullptr) return -4;
   p.kv_mask = a.kv_mask;
   p.N = a.N;
-  p.n_kv = (a.N + kTile - 1) / kTile;
+  p.N_kv = N_kv;
+  p.n_kv = (N_kv + kTile - 1) / kTile;
   if (a.kv_mask != nullptr && p.n_kv > kMaxKvTiles) return -2;
   p.clusters = (a.N + 4 * kTile - 1) / (4 * kTile);
   p.out_f32 = a.out_f32 ? 1 : 0;

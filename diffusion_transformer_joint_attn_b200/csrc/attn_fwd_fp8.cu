@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int wg = warp >> 2;
   if (wg == 1 || wg == 2) {
     const size_t base = static_cast<size_t>(pr.bh) * p.n_blocks;
-    attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.n_kv, p.out_f32, p.scale_log2,
-                       p.q_scale + base, p.k_scale + base, p.n_blocks, nullptr, p.n_kv};
+    attn::SoftmaxIo io{sm.s_full, sm.p_ready, sm.o_final, p.out, p.lse, p.N, p.N, p.n_kv, p.out_f32,
+                       p.scale_log2, p.q_scale + base, p.k_scale + base, p.n_blocks, nullptr, p.n_kv};
     attn::softmax_slot<true>(io, tmem, pr, warp, lane, wc);
   } else {
     if (warp == 0) {

@@ -108,29 +108,73 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
   return cuda_status(dit::launch_prepare_kv(a, static_cast<cudaStream_t>(stream)));
 }
 
+int dit_attn_prepare_kv_split(const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                              void* k_split, void* v_f16, int B, int H, int N, int D, dit_stream_t stream) {
+  if (k == nullptr || v == nullptr || k_split == nullptr || v_f16 == nullptr) return DIT_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * N > (1LL << 40)) return DIT_ERR_INVALID_ARG;
+  if (D != 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_split) || !aligned16(v_f16)) return DIT_ERR_MISALIGNED;
+  if (rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) return DIT_ERR_MISALIGNED;
+  dit::PrepareKVArgs a{k, v, rope_cos, rope_sin, k_split, v_f16, B, H, N, D};
+  return cuda_status(dit::launch_prepare_kv_split(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
 namespace {
 
-// Argument checks and launch shared by the dense and block-sparse entries.
+// Argument checks and launch shared by the dense, key-set and block-sparse
+// entries: N_q queries attend to N_kv keys (N_q == N_kv except for
+// dit_attn_forward_kv).  `kv_tables`: the rotary tables may be applied to k
+// in the kernel (the keys are the query tokens).
 int forward_bf16(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
-                 const uint8_t* kv_mask, void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
-                 dit_stream_t stream) {
+                 const uint8_t* kv_mask, void* out, float* lse, int B, int H, long long N_q, long long N_kv,
+                 bool kv_tables, int D, int dtype, dit_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || N_txt < 0 || N_img < 0) return DIT_ERR_INVALID_ARG;
-  const long long N = static_cast<long long>(N_txt) + N_img;
-  if (N < 1 || N > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
-  if (static_cast<long long>(B) * H > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1) return DIT_ERR_INVALID_ARG;
+  if (N_q < 1 || N_q > 0x7FFFFFFF || N_kv < 1 || N_kv > 0x7FFFFFFF) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x3FFFFFFF) return DIT_ERR_INVALID_ARG;
   if (D != 128) return DIT_ERR_UNSUPPORTED;
-  if ((dtype & ~(DIT_OUT_F32 | DIT_K_ROTATED | DIT_V_F16)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
-  if ((dtype & DIT_K_ROTATED) && rope_cos == nullptr) return DIT_ERR_INVALID_ARG;
-  if (kv_mask != nullptr && N > static_cast<long long>(DIT_SPARSE_MAX_KV_TILES) * 128) return DIT_ERR_UNSUPPORTED;
+  const bool split = (dtype & DIT_QK_SPLIT) != 0;
+  if (split) {
+    // the split form takes the prepared operands of dit_attn_prepare_kv_split
+    if ((dtype & ~(DIT_OUT_F32 | DIT_QK_SPLIT | DIT_V_F16)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+    if (!(dtype & DIT_V_F16)) return DIT_ERR_INVALID_ARG;
+    if (kv_mask != nullptr) return DIT_ERR_UNSUPPORTED;
+  } else {
+    if ((dtype & ~(DIT_OUT_F32 | DIT_K_ROTATED | DIT_V_F16)) != DIT_BF16) return DIT_ERR_UNSUPPORTED;
+    if ((dtype & DIT_K_ROTATED) && rope_cos == nullptr) return DIT_ERR_INVALID_ARG;
+    // tables for the queries only: k must come rotated
+    if (!kv_tables && rope_cos != nullptr && !(dtype & DIT_K_ROTATED)) return DIT_ERR_INVALID_ARG;
+  }
+  if (kv_mask != nullptr && N_kv > static_cast<long long>(DIT_SPARSE_MAX_KV_TILES) * 128) return DIT_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DIT_ERR_MISALIGNED;
   if ((rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) || (lse != nullptr && !aligned4(lse)))
     return DIT_ERR_MISALIGNED;
-  dit::AttnFwdArgs a{q,   k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N), (dtype & DIT_OUT_F32) != 0,
-                     (dtype & DIT_K_ROTATED) != 0, (dtype & DIT_V_F16) != 0, kv_mask};
+  const bool out_f32 = (dtype & DIT_OUT_F32) != 0;
+  if (split) {
+    dit::AttnFwdSplitArgs a{q, k, v, rope_cos, rope_sin, out, lse, B, H, static_cast<int>(N_q), out_f32,
+                            static_cast<int>(N_kv)};
+    return launcher_status(dit::launch_attn_fwd_split(a, static_cast<cudaStream_t>(stream)));
+  }
+  dit::AttnFwdArgs a{q,
+                     k,
+                     v,
+                     rope_cos,
+                     rope_sin,
+                     out,
+                     lse,
+                     B,
+                     H,
+                     static_cast<int>(N_q),
+                     out_f32,
+                     (dtype & DIT_K_ROTATED) != 0,
+                     (dtype & DIT_V_F16) != 0,
+                     kv_mask,
+                     static_cast<int>(N_kv)};
   return launcher_status(dit::launch_attn_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -141,7 +185,15 @@ extern "C" {
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                      void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
                      dit_stream_t stream) {
-  return forward_bf16(q, k, v, rope_cos, rope_sin, nullptr, out, lse, B, H, N_txt, N_img, D, dtype, stream);
+  if (N_txt < 0 || N_img < 0) return DIT_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img;
+  return forward_bf16(q, k, v, rope_cos, rope_sin, nullptr, out, lse, B, H, N, N, true, D, dtype, stream);
+}
+
+int dit_attn_forward_kv(const void* q, const void* k, const void* v, const float* q_cos, const float* q_sin,
+                        void* out, float* lse, int B, int H, int N_q, int N_kv, int D, int dtype,
+                        dit_stream_t stream) {
+  return forward_bf16(q, k, v, q_cos, q_sin, nullptr, out, lse, B, H, N_q, N_kv, false, D, dtype, stream);
 }
 
 size_t dit_attn_forward_host_workspace(int B, int H, int N, int D, int dtype, int chunk_heads) {
@@ -211,7 +263,9 @@ int dit_attn_forward_sparse(const void* q, const void* k, const void* v, const f
                             const float* rope_sin, const uint8_t* kv_mask, void* out, float* lse, int B, int H,
                             int N_txt, int N_img, int D, int dtype, dit_stream_t stream) {
   if (kv_mask == nullptr) return DIT_ERR_INVALID_ARG;
-  return forward_bf16(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, B, H, N_txt, N_img, D, dtype, stream);
+  if (N_txt < 0 || N_img < 0) return DIT_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img;
+  return forward_bf16(q, k, v, rope_cos, rope_sin, kv_mask, out, lse, B, H, N, N, true, D, dtype, stream);
 }
 
 int dit_attn_quantize_fp8(const void* x_bf16, const float* rope_cos, const float* rope_sin, uint8_t* x_fp8,

@@ -28,6 +28,9 @@ struct CopyEngines {
   cudaEvent_t loaded[kBuffers] = {};
   cudaEvent_t computed[kBuffers] = {};
   cudaEvent_t stored[kBuffers] = {};
+  // recorded at the end of each copy stream when an enqueue fails part-way
+  cudaEvent_t h2d_tail = nullptr;
+  cudaEvent_t d2h_tail = nullptr;
 };
 CopyEngines g_engines[kMaxDevices];
 std::mutex g_mu;   // one enqueue sequence at a time (the events are shared)
@@ -38,6 +41,8 @@ cudaError_t engines_for(int dev, CopyEngines** out) {
     cudaError_t r = cudaStreamCreateWithFlags(&e.h2d, cudaStreamNonBlocking);
     if (r == cudaSuccess) r = cudaStreamCreateWithFlags(&e.d2h, cudaStreamNonBlocking);
     if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.start, cudaEventDisableTiming);
+    if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.h2d_tail, cudaEventDisableTiming);
+    if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.d2h_tail, cudaEventDisableTiming);
     for (int b = 0; b < kBuffers && r == cudaSuccess; ++b) {
       r = cudaEventCreateWithFlags(&e.loaded[b], cudaEventDisableTiming);
       if (r == cudaSuccess) r = cudaEventCreateWithFlags(&e.computed[b], cudaEventDisableTiming);
@@ -117,6 +122,14 @@ size_t host_forward_workspace_bytes(int BH, int N, int chunk_heads, bool out_f32
   return kBuffers * buffer_layout(heads, N, out_f32).bytes;
 }
 
+namespace {
+
+// The enqueue sequence of host_forward; on failure it returns at once, leaving
+// whatever it queued on the copy streams.
+cudaError_t host_forward_enqueue(const HostForwardArgs& a, cudaStream_t s, CopyEngines* e);
+
+}  // namespace
+
 cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s) {
   int dev = 0;
   cudaError_t r = cudaGetDevice(&dev);
@@ -125,7 +138,23 @@ cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s) {
   std::lock_guard<std::mutex> lock(g_mu);
   CopyEngines* e = nullptr;
   if ((r = engines_for(dev, &e)) != cudaSuccess) return r;
+  r = host_forward_enqueue(a, s, e);
+  if (r != cudaSuccess) {
+    // An enqueue failed part-way: copies already queued on the private copy
+    // streams still read the caller's host buffers and write its results.
+    // Order them before `stream` (best effort; the first error is the one
+    // returned), so that a caller who synchronises `stream` after the error
+    // may free or reuse those buffers.
+    if (cudaEventRecord(e->h2d_tail, e->h2d) == cudaSuccess) cudaStreamWaitEvent(s, e->h2d_tail, 0);
+    if (cudaEventRecord(e->d2h_tail, e->d2h) == cudaSuccess) cudaStreamWaitEvent(s, e->d2h_tail, 0);
+  }
+  return r;
+}
 
+namespace {
+
+cudaError_t host_forward_enqueue(const HostForwardArgs& a, cudaStream_t s, CopyEngines* e) {
+  cudaError_t r = cudaSuccess;
   const int BH = a.B * a.H;
   const int chunk = std::min(a.chunk_heads, BH);
   const BufferLayout L = buffer_layout(chunk, a.N, a.out_f32);
@@ -198,5 +227,7 @@ cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s) {
     if ((r = cudaStreamWaitEvent(s, e->stored[b], 0)) != cudaSuccess) return r;
   return cudaSuccess;
 }
+
+}  // namespace
 
 }  // namespace dit

@@ -40,6 +40,9 @@ struct PrepareKVArgs {
   int B, H, N, D;
 };
 cudaError_t launch_prepare_kv(const PrepareKVArgs& a, cudaStream_t s);
+// Same arguments; k_rot receives the fp16 split operand [2][B][H][N][D] (hi,
+// then lo) and the tables may be null (no rotation).
+cudaError_t launch_prepare_kv_split(const PrepareKVArgs& a, cudaStream_t s);
 
 struct QuantFp8Args {
   const void* x;       // bf16 [B][H][N][128]
@@ -63,7 +66,8 @@ struct AttnFwdArgs {
   bool out_f32;
   bool k_rotated;   // k already carries the rotary embedding: rotate q only
   bool v_f16;       // v is given as fp16 (otherwise bf16)
-  const uint8_t* kv_mask = nullptr;   // [B*H][ceil(N/512)][ceil(N/128)] block mask, or nullptr (dense)
+  const uint8_t* kv_mask = nullptr;   // [B*H][ceil(N/512)][ceil(N_kv/128)] block mask, or nullptr (dense)
+  int N_kv = 0;     // keys per (b, h) of k and v; 0: N (queries and keys are the same tokens)
 };
 struct AttnFwdFp8Args {
   const void* q8;      // e4m3 [B][H][N][128]
@@ -119,6 +123,22 @@ cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
 // Builds the tensor maps and launches the BF16 forward kernel.
 // Returns 0 on success, a negative dit_status_t otherwise.
 int launch_attn_fwd_bf16(const AttnFwdArgs& a, cudaStream_t s);
+
+// Split (compensated) form: q bf16 rotated and split in the kernel, k the
+// fp16 split operand [2][B][H][N][D] of launch_prepare_kv_split, v fp16.
+struct AttnFwdSplitArgs {
+  const void* q;
+  const void* k_split;
+  const void* v_f16;
+  const float* cos;    // [N][64] or nullptr (no rotary embedding)
+  const float* sin;
+  void* out;
+  float* lse;
+  int B, H, N;
+  bool out_f32;
+  int N_kv = 0;     // keys per (b, h); 0: N
+};
+int launch_attn_fwd_split(const AttnFwdSplitArgs& a, cudaStream_t s);
 
 // cuTensorMapEncodeTiled, resolved once through the runtime's driver entry
 // point (no link-time dependency on libcuda).

@@ -5,10 +5,11 @@
 // 2^x = 2^j * 2^f with j = rint(x) and |f| <= 1/2; 2^f comes from the
 // degree-4 polynomial of least maximum RELATIVE error on [-1/2, 1/2]
 // (2.6e-6 when evaluated in fp32; fitted by fit_exp2_poly.py in this
-// directory), 2^j is added to the exponent field.  x is clamped to >= -126
-// (results there underflow fp16, the format P is stored in, anyway); since
-// the polynomial's value lies in [2^-1/2, 2^1/2], its exponent field stays
-// >= 126 and adding j >= -126 never wraps.
+// directory), 2^j is added to the exponent field.  x is clamped to >= -125
+// (results that small underflow fp16, the format P is stored in, anyway); the
+// polynomial's value lies in [2^-1/2, 2^1/2], so its exponent field is 126 or
+// 127 and adding j >= -125 leaves a field >= 1: the result is always the
+// normal fp32 number p * 2^j.
 // Operates on pairs with Blackwell's packed fp32 add / fma.
 #pragma once
 
@@ -24,8 +25,8 @@ constexpr float kExp2C4 = 9.571337017e-03f;
 constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23: x + magic holds rint(x) in its low mantissa bits
 
 __device__ __forceinline__ void exp2_pair_poly(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
   uint32_t t0, t1;
   float p0, p1;
   asm("{\n\t.reg .b64 x, m, t, j, f, p, c;\n\t"

@@ -62,6 +62,7 @@ typedef enum { DIT_BF16 = 0, DIT_FP8_E4M3 = 1 } dit_dtype_t;
 #define DIT_K_ROTATED 0x200 /* k already carries the rotary embedding (dit_rope_apply); rotate q only */
 #define DIT_V_F16 0x400     /* v is given as fp16 (dit_attn_prepare_kv) instead of bf16 */
 #define DIT_PART_F32 0x800  /* dit_attn_merge: the part outputs are fp32 instead of bf16 */
+#define DIT_QK_SPLIT 0x1000 /* compensated q~ k~^T on fp16 hi + lo operands (dit_attn_prepare_kv_split) */
 #define DIT_SPARSE_MAX_KV_TILES 4096  /* dit_attn_forward_sparse: N <= 4096 x 128 keys */
 #define DIT_MERGE_MAX_PARTS 16
 
@@ -126,6 +127,32 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
                         void* v_f16, int B, int H, int N, int D, dit_stream_t stream);
 
 /*
+ * dit_attn_prepare_kv_split — the operands of the split (compensated) form of
+ * the attention, DIT_QK_SPLIT, prepared once per call in one memory-bound
+ * pass.  That form exists for inputs whose logits are so large that one bf16
+ * rounding of the rotated q and k visibly moves the output: with activation
+ * outliers (channels x16, as modelled for the 2048x2048 workloads) the logits
+ * have a standard deviation of ~45, and the bf16 operand rounding alone moves
+ * O by up to ~7 against exact attention.  The split form keeps such outputs
+ * within the library's BF16 parity bar (max-abs 2e-2, mean-abs 2e-3 against
+ * fp64 attention of the same inputs).
+ *
+ *   k, v      device bf16 [B][H][N][D].
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2] from dit_rope_table_build, or both NULL
+ *             (no rotary embedding).
+ *   k_split   device fp16 [2][B][H][N][D], written: plane 0 holds hi, plane 1
+ *             lo, of r = RN32(RN64(rotated k component)) (both table products
+ *             are exact in fp64): hi = the fp16 nearest r, lo = the fp16
+ *             nearest r - hi, so hi + lo = r to within 2^-22 |r| (2^-25
+ *             absolute where lo is subnormal).  |r| must stay below 65504.
+ *   v_f16     device fp16 [B][H][N][D], written: fp16(v) as dit_attn_prepare_kv.
+ *   B, H, N   >= 1;  D must be 128.  All pointers 16-byte aligned.
+ */
+int dit_attn_prepare_kv_split(const void* k, const void* v, const float* rope_cos, const float* rope_sin,
+                              void* k_split, void* v_f16, int B, int H, int N, int D, dit_stream_t stream);
+
+/*
  * dit_attn_forward — joint attention forward, BF16 in, BF16 (or fp32) out.
  *
  *   q, k, v   device bf16 [B][H][N][D], N = N_txt + N_img.
@@ -145,6 +172,14 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
  *   dtype     DIT_BF16, optionally | DIT_OUT_F32, | DIT_K_ROTATED (requires
  *             the tables: they are then applied to q only) and | DIT_V_F16
  *             (v holds fp16 values, as written by dit_attn_prepare_kv).
+ *             Or the split form: DIT_BF16 | DIT_QK_SPLIT | DIT_V_F16
+ *             [| DIT_OUT_F32], with k the fp16 [2][B][H][N][D] operand and v
+ *             the fp16 values of dit_attn_prepare_kv_split (made with the same
+ *             tables, or none).  The kernel rotates q as that call rotates k,
+ *             splits it into fp16 hi + lo and accumulates
+ *             q~ k~^T = hi_q.lo_k + lo_q.hi_k + hi_q.hi_k in fp32: the logits
+ *             carry ~2^-21 relative error instead of a bf16 operand's 2^-8,
+ *             at three times the tensor-core work of q k^T.
  *
  * Precision: each rotated component of q and k is the bf16 nearest to its
  * exact value for the fp32 table entries; q~ k~^T accumulates in fp32; the
@@ -159,6 +194,36 @@ int dit_attn_prepare_kv(const void* k, const void* v, const float* rope_cos, con
 int dit_attn_forward(const void* q, const void* k, const void* v, const float* rope_cos, const float* rope_sin,
                      void* out, float* lse, int B, int H, int N_txt, int N_img, int D, int dtype,
                      dit_stream_t stream);
+
+/*
+ * dit_attn_forward_kv — dit_attn_forward of N_q queries against a separate
+ * set of N_kv keys and values: one part of key-sharded (context-parallel)
+ * attention, where each part's (out, lse) covers a disjoint key set and
+ * dit_attn_merge combines the parts into the attention over all keys
+ * (wavespeed.ai "Beschleunigung der FLUX.1-dev Bildgenerierung", section on
+ * context parallelism and First Block Cache).
+ *
+ *   q         device bf16 [B][H][N_q][D].
+ *   k, v      device [B][H][N_kv][D] (k bf16, or the fp16 [2][B][H][N_kv][D]
+ *             split operand with DIT_QK_SPLIT; v bf16, or fp16 with DIT_V_F16).
+ *   q_cos, q_sin
+ *             device fp32 [N_q][D/2]: the rotary table rows of the QUERY
+ *             tokens (a contiguous slice of the full table when the queries
+ *             are a contiguous token range), or both NULL.  The kernel rotates
+ *             only q: with tables, k must come rotated (DIT_K_ROTATED, from
+ *             dit_attn_prepare_kv / dit_rope_apply with the key tokens' rows)
+ *             or split (DIT_QK_SPLIT, from dit_attn_prepare_kv_split).
+ *   out, lse  device [B][H][N_q][D] and fp32 [B][H][N_q] (lse may be NULL):
+ *             softmax over the N_kv keys only, and its log-sum-exp.
+ *   N_q, N_kv >= 1.
+ *   dtype     as dit_attn_forward; DIT_K_ROTATED is required when tables are
+ *             given without DIT_QK_SPLIT.
+ * With N_q == N_kv, the same tokens and tables, it returns bit for bit what
+ * dit_attn_forward does.  Same limits, alignment and status handling.
+ */
+int dit_attn_forward_kv(const void* q, const void* k, const void* v, const float* q_cos, const float* q_sin,
+                        void* out, float* lse, int B, int H, int N_q, int N_kv, int D, int dtype,
+                        dit_stream_t stream);
 
 /*
  * dit_attn_forward_host — dit_attn_forward on q, k, v in HOST memory, with
@@ -210,7 +275,12 @@ int dit_attn_forward_host(const void* q, const void* k, const void* v, const flo
  * Arguments, results and status handling as dit_attn_forward_host, minus the
  * workspace.  When dit_attn_forward_host_workspace(B, H, N, D, dtype,
  * chunk_heads) exceeds DIT_STATIC_WORKSPACE_BYTES the call returns
- * DIT_ERR_WORKSPACE and does nothing (fewer heads per chunk need less).
+ * DIT_ERR_WORKSPACE and does nothing.  Fewer heads per chunk need less, but
+ * each of the three chunk buffers holds at least one head (about 1540 N bytes
+ * with bf16 output, 1796 N with fp32), so whatever chunk_heads is, only
+ * N <= DIT_STATIC_MAX_N_BF16_OUT (7262) tokens fit with bf16 output and
+ * N <= DIT_STATIC_MAX_N_F32_OUT (6227) with fp32 output: a 1024x1024 image
+ * (N = 4608) fits, the 2048x2048 (N = 16896) and image-to-image shapes do not.
  * Every call on a device uses the same array: calls that could overlap (from
  * several host threads, or on streams not ordered with each other) race on
  * it and must be serialised by the caller.  The first call on each device
@@ -218,6 +288,8 @@ int dit_attn_forward_host(const void* q, const void* k, const void* v, const flo
  * first call outside any stream capture.
  */
 #define DIT_STATIC_WORKSPACE_BYTES (32u << 20)
+#define DIT_STATIC_MAX_N_BF16_OUT 7262
+#define DIT_STATIC_MAX_N_F32_OUT 6227
 int dit_attn_forward_host_static(const void* q, const void* k, const void* v, const float* rope_cos,
                                  const float* rope_sin, void* out, float* lse, int B, int H, int N_txt, int N_img,
                                  int D, int dtype, int chunk_heads, dit_stream_t stream);

@@ -1,5 +1,5 @@
-"""Number formats used by the oracle: round-to-nearest-even into bf16 and into
-OCP FP8 E4M3 ("e4m3fn": bias 7, largest finite 448, no infinities, NaN is
+"""Number formats used by the oracle: round-to-nearest-even into bf16, fp16,
+fp32 (and the two-term fp16 split of an fp32 value) and into OCP FP8 E4M3 ("e4m3fn": bias 7, largest finite 448, no infinities, NaN is
 S.1111.111), written from the formats' definitions in fp64 arithmetic.
 
 Test infrastructure only (see oracle/__init__.py).
@@ -47,6 +47,26 @@ def round_fp16(x):
     r = _round_nearest_even(x, 11, -14)
     overflow = np.abs(r) > 65504.0
     return np.where(overflow, np.copysign(np.inf, r), r)
+
+
+def round_fp32(x):
+    """Nearest-even IEEE binary32 value of fp64 `x` (24 significand bits,
+    smallest normal 2**-126), returned as fp64; overflow becomes inf."""
+    r = _round_nearest_even(x, 24, -126)
+    fp32_max = (2.0 - 2.0 ** -23) * 2.0 ** 127
+    return np.where(np.abs(r) > fp32_max, np.copysign(np.inf, r), r)
+
+
+def split_fp16(r):
+    """Two-term fp16 representation of fp32 values r (given as fp64):
+    hi = the fp16 nearest r, lo = the fp16 nearest r - hi.  The difference is
+    formed in fp64, where it is exact.  hi + lo is within half an fp16 ulp of
+    lo of r: 2**-22 |r| relative, 2**-25 absolute where lo is subnormal.
+    This is the operand format of the compensated (split) q k^T."""
+    r = np.asarray(r, dtype=np.float64)
+    hi = round_fp16(r)
+    lo = round_fp16(r - hi)
+    return hi, lo
 
 
 def e4m3_decode(codes):

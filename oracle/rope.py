@@ -71,3 +71,14 @@ def rotate_with_table(x, c, s):
     out[..., 0::2] = xe * c - xo * s
     out[..., 1::2] = xe * s + xo * c
     return out
+
+
+def rotate_split(x, c, s):
+    """Operands of the compensated (split) q k^T: the rotation of x [..., N, D]
+    with the table entries c, s [N, D/2], each component evaluated in fp64
+    (both products exact for bf16 x and fp32 entries, the sum rounded once)
+    and rounded to fp32, then split into fp16 hi + lo (formats.split_fp16).
+    Returns (hi, lo) as fp64 arrays of x's shape."""
+    from . import formats
+    r = formats.round_fp32(rotate_with_table(x, c, s))
+    return formats.split_fp16(r)

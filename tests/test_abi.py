@@ -71,6 +71,50 @@ def test_forward_argument_errors(lib):
     assert _fwd(lib, lse=0x70002) == dit.DIT_ERR_MISALIGNED
 
 
+def test_split_form_argument_errors(lib):
+    split = dit.DIT_QK_SPLIT
+    assert _fwd(lib, dtype=split) == dit.DIT_ERR_INVALID_ARG                       # v must be the fp16 operand
+    assert _fwd(lib, dtype=split | dit.DIT_V_F16 | dit.DIT_K_ROTATED) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=split | dit.DIT_V_F16 | dit.DIT_FP8_E4M3) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=split | dit.DIT_V_F16, D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=split | dit.DIT_V_F16, k=0x20004) == dit.DIT_ERR_MISALIGNED
+    # no block-sparse split form
+    assert lib.dit_attn_forward_sparse(0x10000, 0x20000, 0x30000, None, None, 0x9000, 0x40000, None, 1, 1, 8, 8, 128,
+                                       split | dit.DIT_V_F16, None) == dit.DIT_ERR_UNSUPPORTED
+    f = lib.dit_attn_prepare_kv_split
+    ok = dict(k=0x1000, v=0x2000, c=0x3000, s=0x4000, ks=0x5000, vf=0x6000, B=1, H=1, N=8, D=128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["k"], a["v"], a["c"], a["s"], a["ks"], a["vf"], a["B"], a["H"], a["N"], a["D"], None)
+    assert call(k=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(ks=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(s=None) == dit.DIT_ERR_INVALID_ARG                                 # cos without sin
+    assert call(N=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(ks=0x5008) == dit.DIT_ERR_MISALIGNED
+    assert call(c=0x3004) == dit.DIT_ERR_MISALIGNED
+
+
+def test_key_set_forward_argument_errors(lib):
+    f = lib.dit_attn_forward_kv
+
+    def call(q=0x10000, k=0x20000, cos=None, sin=None, Nq=8, Nkv=16, D=128, dtype=0, lse=None):
+        return f(q, k, 0x30000, cos, sin, 0x40000, lse, 1, 2, Nq, Nkv, D, dtype, None)
+    assert call(q=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(Nq=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(Nkv=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(Nkv=-5) == dit.DIT_ERR_INVALID_ARG
+    assert call(cos=0x50000) == dit.DIT_ERR_INVALID_ARG                            # sin missing
+    # the tables rotate q only: k must come rotated (or split)
+    assert call(cos=0x50000, sin=0x60000) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(dtype=0x800) == dit.DIT_ERR_UNSUPPORTED
+    assert call(q=0x10008) == dit.DIT_ERR_MISALIGNED
+    assert call(lse=0x70002) == dit.DIT_ERR_MISALIGNED
+    assert call(cos=0x50000, sin=0x60000, dtype=dit.DIT_QK_SPLIT) == dit.DIT_ERR_INVALID_ARG   # v fp16 required
+
+
 def test_sparse_forward_argument_errors(lib):
     f = lib.dit_attn_forward_sparse
 
@@ -115,6 +159,20 @@ def test_static_workspace_entry_rejects_oversize_without_a_gpu(lib):
                                           0, 4, None)
     assert rc == dit.DIT_ERR_WORKSPACE
     assert dit.dit_attn_status_string(rc) == "problem needs more workspace than the static workspace holds"
+
+
+def test_static_workspace_token_limit_at_one_head_per_chunk(lib):
+    """The header's largest N for the static workspace holds at chunk_heads = 1,
+    the smallest chunk: N fits, N + 1 does not (bf16 and fp32 output)."""
+    size = lib.dit_attn_forward_host_workspace
+    for dtype, n_max in ((dit.DIT_BF16, 7262), (dit.DIT_BF16 | dit.DIT_OUT_F32, 6227)):
+        assert size(1, 1, n_max, 128, dtype, 1) <= 32 << 20
+        assert size(1, 1, n_max + 1, 128, dtype, 1) > 32 << 20
+        # one head per chunk is the minimum whatever chunk_heads asks for
+        assert size(1, 24, n_max + 1, 128, dtype, 1) > 32 << 20
+        rc = lib.dit_attn_forward_host_static(0x1000, 0x2000, 0x3000, None, None, 0x4000, None, 1, 24, 0,
+                                              n_max + 1, 128, dtype, 1, None)
+        assert rc == dit.DIT_ERR_WORKSPACE
 
 
 def test_static_workspace_entry_argument_errors_before_any_cuda_call(lib):

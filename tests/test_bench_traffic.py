@@ -15,10 +15,16 @@ CSRC = os.path.join("diffusion_transformer_joint_attn_b200", "csrc")
 
 
 def _copy_tree(tmp_path):
-    """A copy of the kernel sources and the traffic record under tmp_path."""
+    """A copy of the kernel sources under tmp_path with a traffic record whose
+    hashes match them (whether or not the committed record is current)."""
     shutil.copytree(os.path.join(ROOT, CSRC), tmp_path / CSRC)
     (tmp_path / "profiles").mkdir()
-    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    for kernel in bench.KERNEL_SOURCES:
+        rec["kernels"][kernel]["source_sha"] = bench.kernel_source_sha(kernel)
+    with open(tmp_path / "profiles" / "traffic.json", "w") as f:
+        json.dump(rec, f)
     return tmp_path
 
 

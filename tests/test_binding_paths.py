@@ -77,6 +77,34 @@ def test_forward_wrappers():
                                                       stream=0))
 
 
+def test_split_and_key_set_wrappers():
+    q = OnGpu((B, H, N, D), bf16)
+    c, s = OnGpu((N, 64), f32), OnGpu((N, 64), f32)
+    k_split, v16 = OnGpu((2, B, H, N, D), f16), OnGpu((B, H, N, D), f16)
+    fails_at_cuda(lambda: dit.dit_attn_prepare_kv_split(q, q, c, s, k_split, v16, stream=0))
+    fails_at_cuda(lambda: dit.dit_attn_prepare_kv_split(q, q, None, None, k_split, v16, stream=0))
+    out, lse = OnGpu((B, H, N, D), f32), OnGpu((B, H, N), f32)
+    fails_at_cuda(lambda: dit.dit_attn_forward(q, k_split, v16, c, s, out, lse, NT, NI,
+                                               dit.DIT_QK_SPLIT | dit.DIT_V_F16 | dit.DIT_OUT_F32, stream=0))
+    with pytest.raises(ValueError, match="DIT_QK_SPLIT"):    # a bf16 k is not the split operand
+        dit.dit_attn_forward(q, q, v16, c, s, out, lse, NT, NI, dit.DIT_QK_SPLIT | dit.DIT_V_F16 | dit.DIT_OUT_F32,
+                             stream=0)
+    # queries of tokens 0..N-1 against a shard of 40 keys
+    Nkv = 40
+    kr, vk = OnGpu((B, H, Nkv, D), bf16), OnGpu((B, H, Nkv, D), f16)
+    fails_at_cuda(lambda: dit.dit_attn_forward_kv(q, kr, vk, c, s, out, lse,
+                                                  dit.DIT_K_ROTATED | dit.DIT_V_F16 | dit.DIT_OUT_F32, stream=0))
+    ks = OnGpu((2, B, H, Nkv, D), f16)
+    fails_at_cuda(lambda: dit.dit_attn_forward_kv(q, ks, vk, c, s, out, None,
+                                                  dit.DIT_QK_SPLIT | dit.DIT_V_F16 | dit.DIT_OUT_F32, stream=0))
+    with pytest.raises(ValueError, match="N_kv"):
+        dit.dit_attn_forward_kv(q, OnGpu((B, H, Nkv + 1, D), bf16), vk, c, s, out, lse,
+                                dit.DIT_K_ROTATED | dit.DIT_V_F16 | dit.DIT_OUT_F32, stream=0)
+    with pytest.raises(ValueError, match="rope tables"):     # the query tables have N_q rows
+        dit.dit_attn_forward_kv(q, kr, vk, OnGpu((Nkv, 64), f32), OnGpu((Nkv, 64), f32), out, lse,
+                                dit.DIT_K_ROTATED | dit.DIT_V_F16 | dit.DIT_OUT_F32, stream=0)
+
+
 def test_fp8_wrappers():
     x = OnGpu((B, H, N, D), bf16)
     codes, scale = OnGpu((B, H, N, D), u8), OnGpu((B, H, 1), f32)

@@ -115,3 +115,35 @@ def test_tie_count_finds_constructed_ties():
     scales = fp8.block_scales(x)
     assert scales[0, 0] == 1.0
     assert fp8.tie_count(x, scales) == 1
+
+
+def test_round_fp32_matches_library_cast_and_ties_to_even():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(200000) * np.exp(rng.uniform(-95, 85, 200000))
+    assert np.array_equal(formats.round_fp32(x), x.astype(np.float32).astype(np.float64))
+    ulp = 2.0 ** -23
+    assert formats.round_fp32(1.0 + ulp / 2) == 1.0
+    assert formats.round_fp32(1.0 + 1.5 * ulp) == 1.0 + 2 * ulp
+    assert formats.round_fp32(2.0 ** -140 * 1.25) == np.float64(np.float32(2.0 ** -140 * 1.25))   # subnormal
+    assert formats.round_fp32(4.0e38) == np.inf
+
+
+def test_split_fp16_terms():
+    rng = np.random.default_rng(6)
+    r = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 10, 100000))).astype(np.float32).astype(np.float64)
+    hi, lo = formats.split_fp16(r)
+    # hi is the library's fp16 cast of r; lo the cast of the exact remainder
+    assert np.array_equal(hi, _torch_round(r, torch.float16))
+    assert np.array_equal(lo, _torch_round(r - hi, torch.float16))
+    # hi + lo carries r to 2^-22 relative (2^-25 absolute once lo is subnormal)
+    assert np.all(np.abs(hi + lo - r) <= np.maximum(2.0 ** -22 * np.abs(r), 2.0 ** -25))
+    # the remainder is at most half an fp16 ulp of hi
+    assert np.all(np.abs(r - hi) <= np.ldexp(1.0, np.frexp(np.abs(hi))[1] - 12) + 2.0 ** -25)
+    # worked cases: exactly representable, a remainder one fp16 ulp below, a subnormal remainder
+    assert formats.split_fp16(0.75) == (0.75, 0.0)
+    assert formats.split_fp16(1.0 + 2.0 ** -15) == (1.0, 2.0 ** -15)
+    assert formats.split_fp16(1.0 + 2.0 ** -21) == (1.0, 2.0 ** -21)
+    # remainder 1.5 * 2^-24 lies halfway between the fp16 subnormals 2^-24 and 2^-23: the even one is taken
+    h, l = formats.split_fp16(2.0 ** -12 + 1.5 * 2.0 ** -24)
+    assert h == 2.0 ** -12 and l == 2.0 ** -23
+    assert formats.split_fp16(-3.0 - 2.0 ** -14) == (-3.0, -(2.0 ** -14))

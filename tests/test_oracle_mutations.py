@@ -79,7 +79,25 @@ def _round_half_up(x, sig_bits, min_exp):
     return np.sign(x) * np.floor(ax / step + 0.5) * step             # ties away from zero
 
 
-_ORIG = {"frequencies": rope.frequencies, "attention_rows": attention.attention_rows, "merge": merge.merge,
+def _split_remainder_unrounded(r):
+    hi = _ORIG["round_fp16"](np.asarray(r, dtype=np.float64))
+    return hi, np.asarray(r, dtype=np.float64) - hi                   # lo not rounded to fp16
+
+
+def _split_truncated(r):
+    r = np.asarray(r, dtype=np.float64)
+    _, e = np.frexp(np.abs(r))
+    step = np.ldexp(1.0, np.maximum(e - 1, -14) - 10)
+    hi = np.trunc(r / step) * step                                    # hi chopped instead of rounded
+    return hi, _ORIG["round_fp16"](r - hi)
+
+
+def _fp32_chopped(x):
+    x = np.asarray(x, dtype=np.float64)
+    return x.astype(np.float32).astype(np.float64) * (1.0 - 2.0 ** -24)
+
+
+_ORIG = {"round_fp16": formats.round_fp16, "frequencies": rope.frequencies, "attention_rows": attention.attention_rows, "merge": merge.merge,
          "block_scales": fp8.block_scales}
 
 # pins, as callables without arguments
@@ -90,6 +108,7 @@ P_ROPE = [TA.test_rope_rotation_direction, TA.test_rope_relative_position,
 P_ATTN = [TA.test_rows_sum_to_one, TA.test_zero_query_gives_column_mean_and_log_n,
           TA.test_dominant_key_returns_its_value_row, lambda: TA.test_matches_library_sdpa_without_rope(64)]
 P_MERGE = [TA.test_merge_of_key_slices_equals_full_attention, TA.test_merge_weights_follow_the_softmax_of_the_lses]
+P_SPLIT = [TF.test_split_fp16_terms, TF.test_round_fp32_matches_library_cast_and_ties_to_even]
 P_FP8 = [TF.test_block_quantisation_properties, TF.test_e4m3_midpoints_round_to_even_and_saturate,
          TF.test_e4m3_encode_matches_library_cast, TF.test_e4m3_landmark_codes]
 
@@ -104,6 +123,9 @@ MUTATIONS = [
     ("merge not renormalised", merge, "merge", _merge_unnormalised, P_MERGE),
     ("E4M3 scale from 240", fp8, "block_scales", _fp8_max_240, P_FP8),
     ("rounding ties away from zero", formats, "_round_nearest_even", _round_half_up, P_FP8),
+    ("split remainder not rounded", formats, "split_fp16", _split_remainder_unrounded, P_SPLIT),
+    ("split hi chopped", formats, "split_fp16", _split_truncated, P_SPLIT),
+    ("fp32 rounding biased", formats, "round_fp32", _fp32_chopped, P_SPLIT),
 ]
 
 
@@ -120,5 +142,5 @@ def test_planted_mistake_fails_a_pin(name, module, attr, bad, pins, monkeypatch)
 
 
 def test_pins_pass_on_the_unmodified_oracle():
-    for pin in P_BRUTE + P_ROPE + P_ATTN + P_MERGE + P_FP8:
+    for pin in P_BRUTE + P_ROPE + P_ATTN + P_MERGE + P_FP8 + P_SPLIT:
         pin()

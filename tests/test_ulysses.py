@@ -69,10 +69,13 @@ def _worker(rank, world, port, case, rq):
             result["tables"] = refused(lambda: ulysses.ulysses_attention(
                 shard, shard, shard, torch.zeros(4, 64), torch.zeros(4, 64), attn=lambda *a: None))
             result["shapes"] = refused(lambda: ulysses.ulysses_attention(shard, shard[:, :1], shard))
+            result["groups"] = refused(lambda: ulysses.ulysses_attention(shard, shard, shard, head_groups=3,
+                                                                         attn=lambda *a: None))
             dist.barrier()                        # the ranks are still in step
         else:
             import workloads as W
             from oracle import attention as oracle_attention
+            head_groups = 3 if case == "grouped" else 1
             cfg_groups = 2 if case == "cfg" else 1
             groups = ulysses.cfg_ulysses_groups(world, cfg_groups)
             handles = [dist.new_group(r) for r in groups]          # every rank creates every group, in order
@@ -80,7 +83,7 @@ def _worker(rank, world, port, case, rq):
             group = handles[gi]
             P = world // cfg_groups
             r_in = rank % P
-            w = W.custom(2 if case == "cfg" else 1, 2 * P, 8 * P, ((4 * P, 6),))
+            w = W.custom(2 if case == "cfg" else 1, 2 * P * head_groups, 8 * P, ((4 * P, 6),))
             q, k, v = W.make_qkv(w, seed=3)
             pos = W.positions(w)
             share = ulysses.batch_share(w.B, gi, cfg_groups)
@@ -95,8 +98,14 @@ def _worker(rank, world, port, case, rq):
                 return (torch.from_numpy(O.reshape(Bl, Hl, N, -1)), torch.from_numpy(L.reshape(Bl, Hl, N)))
 
             cs = torch.zeros(w.N, 64)             # tables of all N tokens (the oracle uses pos)
+            calls = []
+
+            def counted(*a):
+                calls.append(a[0].shape[1])
+                return oracle_attn(*a)
             out, lse = ulysses.ulysses_attention(local(q), local(k), local(v), cs, cs, n_txt=w.n_txt, group=group,
-                                                 attn=oracle_attn)
+                                                 attn=counted, head_groups=head_groups)
+            result["attn_calls"] = calls
             O, L = oracle_attention.joint_attention(q, k, v, pos=pos)
             O = O.reshape(w.B, w.H, w.N, -1)[share, :, r_in * Ns:(r_in + 1) * Ns]
             L = L.reshape(w.B, w.H, w.N)[share, :, r_in * Ns:(r_in + 1) * Ns]
@@ -135,6 +144,16 @@ def test_ulysses_attention_matches_full_sequence_oracle(world):
     res = _run(world, "ulysses")
     for rank, r in res.items():
         assert r["max_err"] < 1e-12 and r["lse_err"] < 1e-12, (rank, r)
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_group_pipelined_exchanges_match_full_sequence_oracle(world):
+    """Three head groups per rank: three attention calls of 2 heads each, and
+    the result of the whole-tensor exchange."""
+    res = _run(world, "grouped")
+    for rank, r in res.items():
+        assert r["max_err"] < 1e-12 and r["lse_err"] < 1e-12, (rank, r)
+        assert r["attn_calls"] == [2, 2, 2], (rank, r)
 
 
 def test_exchange_argument_errors_on_every_rank():
