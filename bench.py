@@ -374,6 +374,42 @@ def time_split(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev):
                          "work": "tensor work 8 N^2 D H B per launch (q k^T x3 + P V), twice the method's count"}}
 
 
+def time_projection(args, w, lib, cos, sin, stream, dev, C=3072):
+    """dit_qkv_project_fp8 on the workload's token count: the QKV projection
+    of seeded hidden states x [B, N, 3072] (the FLUX width, 24 heads x 128)
+    with a seeded weight [3 H 128, 3072], the rotary embedding of q, k and the
+    E4M3 block quantisation of q, k, v in its epilogue.  A GEMM of 2 B N C
+    (3 H 128) FLOP; its roofline is the tensor peak."""
+    import torch
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(w.B, w.N, C, generator=g).to(torch.bfloat16).to(dev)
+    wt = (torch.randn(3 * w.H * 128, C, generator=g) / C ** 0.5).to(torch.bfloat16).to(dev)
+    bias = (0.1 * torch.randn(3 * w.H * 128, generator=g)).float().to(dev)
+    nb = (w.N + 63) // 64
+    codes = [torch.empty((w.B, w.H, w.N, 128), dtype=torch.uint8, device=dev) for _ in range(3)]
+    scales = [torch.empty((w.B, w.H, nb), dtype=torch.float32, device=dev) for _ in range(3)]
+    s_ptr = stream.cuda_stream
+
+    def launch():
+        assert lib.dit_qkv_project_fp8(x.data_ptr(), wt.data_ptr(), bias.data_ptr(), cos.data_ptr(), sin.data_ptr(),
+                                       *[t.data_ptr() for t in codes], *[t.data_ptr() for t in scales], None, None,
+                                       None, w.B, w.N, C, w.H, 128, s_ptr) == 0
+
+    ms = statistics.mean(time_launches(launch, stream, dev, max(1, min(args.steps, 20))))
+    import diffusion_transformer_joint_attn_b200 as dit
+    if dit.dit_attn_get_status(stream) != 0:
+        raise RuntimeError("device status error in the projection timing")
+    flops = 2.0 * w.B * w.N * C * 3 * w.H * 128
+    peak, src = measured_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"kernel_ms": ms, "value": achieved, "unit": UNIT, "tflop_per_launch": flops / 1e12,
+            "shape": "x [%d, %d, %d] x w [%d, %d]" % (w.B, w.N, C, 3 * w.H * 128, C),
+            "step": "QKV projection GEMM with rotary embedding and E4M3 block quantisation in its epilogue",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "kernel": "qkv_proj_fp8_kernel", "traffic": None,
+                         "peak_source": src}}
+
+
 def time_fused_k(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev):
     """The forward with the rotary embedding of K inside the kernel's tile
     prologue (raw bf16 K and V: each query tile's CTA pair rotates every K
@@ -574,6 +610,7 @@ def run_native(args):
     median50 = statistics.median(time_launches(attn_launch, stream, dev, 50))
     split = time_split(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev)
     fused_k = time_fused_k(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev)
+    proj = time_projection(args, w, lib, cos, sin, stream, dev)
     sdpa = time_sdpa_context(args, w, q, k, v, stream, dev)
 
     # end to end through the public C ABI with host buffers: pinned q, k, v
@@ -656,6 +693,7 @@ def run_native(args):
             "fp8": fp8,
             "split": split,
             "fused_k": fused_k,
+            "qkv_projection": proj,
             "merge": merge,
             "sparse": sparse,
             "context_library_sdpa": sdpa,

@@ -312,6 +312,39 @@ def dit_attn_forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, n_txt:
                                                _stream(stream)), "dit_attn_forward_fp8")
 
 
+def dit_qkv_project_fp8(x, w, bias, rope_cos, rope_sin, q8, k8, v8, q_scale, k_scale, v_scale, q16=None, k16=None,
+                        v16=None, stream=None) -> None:
+    """E4M3 codes and block scales of the rotated q, k and of v (and optionally the bf16 q, k, v) from the QKV
+    projection of the hidden states x [B, N, C] (bf16) with the weight w [3 H 128, C] (bf16) and an optional fp32
+    bias [3 H 128]."""
+    import torch
+    _require(x.dim() == 3 and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous(),
+             "x must be a contiguous CUDA bf16 [B, N, C] tensor")
+    B, N, C = x.shape
+    _require(w.dim() == 2 and w.shape[1] == C and w.shape[0] % 384 == 0 and w.is_cuda and w.dtype == torch.bfloat16
+             and w.is_contiguous(), "w must be a contiguous CUDA bf16 [3 H 128, C] tensor")
+    H = w.shape[0] // 384
+    if bias is not None:
+        _require(bias.is_cuda and bias.dtype == torch.float32 and bias.is_contiguous() and
+                 tuple(bias.shape) == (w.shape[0],), "bias must be a contiguous CUDA fp32 [3 H 128] tensor")
+    _check_tables(rope_cos, rope_sin, N, 128)
+    for t in (q8, k8, v8):
+        _require(t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous() and tuple(t.shape) == (B, H, N, 128),
+                 "q8, k8, v8 must be contiguous CUDA uint8 [B, H, N, 128] tensors")
+    for t in (q_scale, k_scale, v_scale):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                 tuple(t.shape) == (B, H, (N + 63) // 64), "scales must be contiguous CUDA fp32 [B, H, ceil(N/64)]")
+    for t in (q16, k16, v16):
+        if t is not None:
+            _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and
+                     tuple(t.shape) == (B, H, N, 128), "q16, k16, v16 must be contiguous CUDA bf16 [B, H, N, 128]")
+    _on_current_device(x, w, bias, rope_cos, rope_sin, q8, k8, v8, q_scale, k_scale, v_scale, q16, k16, v16)
+    _check(load_library().dit_qkv_project_fp8(_ptr(x), _ptr(w), _ptr(bias), _ptr(rope_cos), _ptr(rope_sin), _ptr(q8),
+                                              _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+                                              _ptr(q16), _ptr(k16), _ptr(v16), B, N, C, H, 128, _stream(stream)),
+           "dit_qkv_project_fp8")
+
+
 def dit_attn_merge(o_parts, lse_parts, out, lse_out=None, dtype: int = DIT_BF16, stream=None) -> None:
     """out (and lse_out) <- merge of R partial results (lists of [B, H, N, D] outputs and [B, H, N] lses)
     over disjoint key sets."""
@@ -398,6 +431,20 @@ def forward_kv(q, k, v, q_cos=None, q_sin=None, out_f32: bool = False, with_lse:
     dit_attn_forward_kv(q, k, v, q_cos, q_sin, out, lse, DIT_BF16 | _flags(out_f32, k_rotated, v_f16 or qk_split,
                                                                         qk_split), stream)
     return out, lse
+
+
+def qkv_project_fp8(x, w, bias=None, rope_cos=None, rope_sin=None, with_bf16: bool = False, stream=None):
+    """Allocate and fill the FP8 attention operands from the QKV projection of x [B, N, C] with w [3 H 128, C]:
+    returns (q8, k8, v8, q_scale, k_scale, v_scale, q16, k16, v16); the bf16 tensors are None unless with_bf16."""
+    import torch
+    B, N, _ = x.shape
+    H = w.shape[0] // 384
+    codes = [torch.empty((B, H, N, 128), dtype=torch.uint8, device=x.device) for _ in range(3)]
+    scales = [torch.empty((B, H, (N + 63) // 64), dtype=torch.float32, device=x.device) for _ in range(3)]
+    y16 = [torch.empty((B, H, N, 128), dtype=torch.bfloat16, device=x.device) if with_bf16 else None
+           for _ in range(3)]
+    dit_qkv_project_fp8(x, w, bias, rope_cos, rope_sin, *codes, *scales, *y16, stream=stream)
+    return (*codes, *scales, *y16)
 
 
 def merge(o_parts, lse_parts, out_f32: bool = False, with_lse: bool = True, stream=None):

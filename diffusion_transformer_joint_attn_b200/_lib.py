@@ -27,6 +27,7 @@ SIGNATURES = {
     "dit_attn_forward_sparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_quantize_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "dit_attn_forward_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
+    "dit_qkv_project_fp8": (_I, [_VP] * 14 + [_I, _I, _I, _I, _I, _VP]),
     "dit_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     "dit_attn_wait_selftest": (_I, [ctypes.c_longlong, _VP]),
     "dit_attn_get_status": (_I, [ctypes.POINTER(ctypes.c_int), _VP]),

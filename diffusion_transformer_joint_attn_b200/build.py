@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libdit_attn.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["capi.cu", "rope_table.cu", "rope_apply.cu", "quant_fp8.cu", "attn_fwd.cu", "attn_fwd_split.cu", "attn_fwd_fp8.cu", "merge.cu", "host_pipeline.cu", "wait_selftest.cu"]
+SOURCES = ["capi.cu", "rope_table.cu", "rope_apply.cu", "quant_fp8.cu", "attn_fwd.cu", "attn_fwd_split.cu", "attn_fwd_fp8.cu", "merge.cu", "qkv_proj.cu", "host_pipeline.cu", "wait_selftest.cu"]
 
 
 def nvcc_path() -> str:

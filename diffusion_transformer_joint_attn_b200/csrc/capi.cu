@@ -300,6 +300,30 @@ int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8
   return launcher_status(dit::launch_attn_fwd_fp8(a, static_cast<cudaStream_t>(stream)));
 }
 
+int dit_qkv_project_fp8(const void* x, const void* w, const float* bias, const float* rope_cos,
+                        const float* rope_sin, uint8_t* q8, uint8_t* k8, uint8_t* v8, float* q_scale, float* k_scale,
+                        float* v_scale, void* q16, void* k16, void* v16, int B, int N, int C, int H, int D,
+                        dit_stream_t stream) {
+  if (x == nullptr || w == nullptr || q8 == nullptr || k8 == nullptr || v8 == nullptr || q_scale == nullptr ||
+      k_scale == nullptr || v_scale == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || C < 1 || H < 1) return DIT_ERR_INVALID_ARG;
+  if (B > 65535 || static_cast<long long>(B) * H * N * 128 > (1LL << 40) || static_cast<long long>(C) * N * B > (1LL << 40))
+    return DIT_ERR_INVALID_ARG;
+  if (D != 128 || (H & 1) || (C & 7)) return DIT_ERR_UNSUPPORTED;
+  const void* out16[3] = {q16, k16, v16};
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8)) return DIT_ERR_MISALIGNED;
+  if (!aligned4(q_scale) || !aligned4(k_scale) || !aligned4(v_scale) || (bias != nullptr && !aligned4(bias)))
+    return DIT_ERR_MISALIGNED;
+  if (rope_cos != nullptr && (!aligned16(rope_cos) || !aligned16(rope_sin))) return DIT_ERR_MISALIGNED;
+  for (const void* o : out16)
+    if (o != nullptr && !aligned16(o)) return DIT_ERR_MISALIGNED;
+  dit::QkvProjArgs a{x,  w,  bias, rope_cos, rope_sin, {q8, k8, v8}, {q_scale, k_scale, v_scale},
+                     {q16, k16, v16}, B, N, C, H};
+  return launcher_status(dit::launch_qkv_proj_fp8(a, static_cast<cudaStream_t>(stream)));
+}
+
 static_assert(DIT_MERGE_MAX_PARTS == dit::kMergeMaxParts, "part limit of the header and the kernel differ");
 static_assert(DIT_STATIC_WORKSPACE_BYTES == dit::kStaticWorkspaceBytes, "static workspace size differs");
 

@@ -117,6 +117,20 @@ constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
 cudaError_t static_workspace(void** out);
 cudaError_t host_forward(const HostForwardArgs& a, cudaStream_t s);
 
+// QKV projection with the FP8 operand epilogue (qkv_proj.cu).
+struct QkvProjArgs {
+  const void* x;         // bf16 [B][N][C]
+  const void* w;         // bf16 [3 H 128][C]
+  const float* bias;     // [3 H 128] or nullptr
+  const float* cos;      // [N][64] or nullptr (no rotary embedding)
+  const float* sin;
+  uint8_t* codes[3];     // q8, k8, v8 [B][H][N][128]
+  float* scales[3];      // [B][H][ceil(N/64)]
+  void* y16[3];          // bf16 q, k, v [B][H][N][128] or nullptr
+  int B, N, C, H;
+};
+int launch_qkv_proj_fp8(const QkvProjArgs& a, cudaStream_t s);
+
 // Bounded-wait self-test (wait_selftest.cu).
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
 

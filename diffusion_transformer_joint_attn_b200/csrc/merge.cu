@@ -9,7 +9,8 @@
 // its O_r are not used; a row whose parts are all empty gets O = 0 and lse = -inf.
 //
 // Memory-bound: 16 threads per row, 8 channels (one 16-byte bf16 or two
-// 16-byte fp32 loads per part) each, every load of a row in flight at once;
+// 16-byte fp32 loads per part) each; every load of a row, and those of the
+// group's next row, are in flight at once;
 // the parts are read through plain global loads, so they may live in a peer
 // GPU's memory mapped into this context.
 #include <cuda_bf16.h>
@@ -67,26 +68,46 @@ __device__ __forceinline__ void unpack(const Chunk<kInF32>& c, float* v) {
   }
 }
 
+// One row's loads: R lses and R output chunks (parts past R read as empty).
+template <int kR, bool kInF32>
+struct RowLoads {
+  float l[kR];
+  Chunk<kInF32> c[kR];
+};
+
+template <int kR, bool kInF32>
+__device__ __forceinline__ void load_row(const MergeParams& p, long long row, int sub, RowLoads<kR, kInF32>& x) {
+#pragma unroll
+  for (int r = 0; r < kR; ++r) {
+    if (r < p.R && row < p.rows) {
+      x.l[r] = __ldg(p.lse[r] + row);
+      x.c[r] = load_chunk<kInF32>(p.o[r], row, sub);
+    } else {
+      x.l[r] = -INFINITY;
+    }
+  }
+}
+
 // kR: parts this instantiation holds in registers (R <= kR).  All loads of a
-// row (R lses, R output chunks) are issued before the first is used.
+// row (R lses, R output chunks) are issued before the first is used; with up
+// to 4 parts the loads of the group's next row are issued too before this
+// row is combined (with more parts the registers would spill).
 template <int kR, bool kInF32, bool kOutF32>
 __global__ void __launch_bounds__(kThreads) merge_kernel(const MergeParams p) {
+  constexpr bool kPrefetch = kR <= 4;
   const int sub = threadIdx.x % kLanesPerRow;
   const unsigned half_mask = 0xFFFFu << (threadIdx.x & 16);
   const long long stride = static_cast<long long>(gridDim.x) * kRowsPerBlock;
-  for (long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanesPerRow;
-       row < p.rows; row += stride) {
-    float l[kR];
-    Chunk<kInF32> c[kR];
-#pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      if (r < p.R) {
-        l[r] = __ldg(p.lse[r] + row);
-        c[r] = load_chunk<kInF32>(p.o[r], row, sub);
-      } else {
-        l[r] = -INFINITY;
-      }
-    }
+  long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kLanesPerRow;
+  RowLoads<kR, kInF32> cur, nxt;
+  if (kPrefetch) load_row<kR, kInF32>(p, row, sub, cur);
+  for (; row < p.rows; row += stride) {
+    if (kPrefetch)
+      load_row<kR, kInF32>(p, row + stride, sub, nxt);
+    else
+      load_row<kR, kInF32>(p, row, sub, cur);
+    const float* l = cur.l;
+    const Chunk<kInF32>* c = cur.c;
     float m = -INFINITY;
 #pragma unroll
     for (int r = 0; r < kR; ++r) m = fmaxf(m, l[r]);
@@ -127,22 +148,29 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const MergeParams p) {
           make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (sub == 0 && p.lse_out != nullptr) p.lse_out[row] = empty ? -INFINITY : m + logf(total);
+    if (kPrefetch) cur = nxt;
   }
 }
 
+// A grid-stride launch of the instance with exactly the CTAs that are
+// resident at once (the rows are split evenly over them).
+template <int kR, bool kInF32, bool kOutF32>
+cudaError_t launch_one(const MergeParams& p, long long need, cudaStream_t s) {
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, merge_kernel<kR, kInF32, kOutF32>,
+                                                                      kThreads, 0);
+  if (r != cudaSuccess) return r;
+  const long long cap = static_cast<long long>(sms) * (per_sm > 0 ? per_sm : 1);
+  merge_kernel<kR, kInF32, kOutF32><<<static_cast<unsigned>(need < cap ? need : cap), kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
 template <int kR>
-void launch_bucket(const MergeParams& p, bool in_f32, bool out_f32, unsigned grid, cudaStream_t s) {
-  if (in_f32) {
-    if (out_f32)
-      merge_kernel<kR, true, true><<<grid, kThreads, 0, s>>>(p);
-    else
-      merge_kernel<kR, true, false><<<grid, kThreads, 0, s>>>(p);
-  } else {
-    if (out_f32)
-      merge_kernel<kR, false, true><<<grid, kThreads, 0, s>>>(p);
-    else
-      merge_kernel<kR, false, false><<<grid, kThreads, 0, s>>>(p);
-  }
+cudaError_t launch_bucket(const MergeParams& p, bool in_f32, bool out_f32, long long need, cudaStream_t s) {
+  if (in_f32)
+    return out_f32 ? launch_one<kR, true, true>(p, need, s) : launch_one<kR, true, false>(p, need, s);
+  return out_f32 ? launch_one<kR, false, true>(p, need, s) : launch_one<kR, false, false>(p, need, s);
 }
 
 }  // namespace
@@ -157,20 +185,11 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
   p.lse_out = a.lse_out;
   p.rows = a.rows;
   p.R = a.R;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long need = (a.rows + kRowsPerBlock - 1) / kRowsPerBlock;
-  const long long cap = static_cast<long long>(sms) * (2048 / kThreads);
-  const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
-  if (a.R <= 2)
-    launch_bucket<2>(p, a.in_f32, a.out_f32, grid, s);
-  else if (a.R <= 4)
-    launch_bucket<4>(p, a.in_f32, a.out_f32, grid, s);
-  else if (a.R <= 8)
-    launch_bucket<8>(p, a.in_f32, a.out_f32, grid, s);
-  else
-    launch_bucket<16>(p, a.in_f32, a.out_f32, grid, s);
-  return cudaGetLastError();
+  if (a.R <= 2) return launch_bucket<2>(p, a.in_f32, a.out_f32, need, s);
+  if (a.R <= 4) return launch_bucket<4>(p, a.in_f32, a.out_f32, need, s);
+  if (a.R <= 8) return launch_bucket<8>(p, a.in_f32, a.out_f32, need, s);
+  return launch_bucket<16>(p, a.in_f32, a.out_f32, need, s);
 }
 
 }  // namespace dit

@@ -1,0 +1,315 @@
+// The QKV projection of the joint token sequence with the FP8 operand
+// preparation fused into its epilogue (sm_100a).
+//
+//   y[b, n, o] = sum_c x[b, n, c] w[o, c] (+ bias[o]),  o = s H D + h D + d
+//
+// is a bf16 x bf16 -> fp32 GEMM on the tensor cores (tcgen05, accumulator
+// in tensor memory).  Its epilogue turns the accumulator tile straight into
+// the operands of dit_attn_forward_fp8, with no round trip of y through
+// HBM: for q and k it applies the rotary embedding (each pair turned in
+// fp64 from the fp32 accumulator and the fp32 table entries, rounded to
+// fp32), takes the amax of every block of 64 tokens x 128 channels of one
+// (b, h), and writes the E4M3 codes of y / (amax / 448) and the block scale;
+// optionally also the unrotated y rounded to bf16 in the attention layout.
+//
+// One CTA per tile of 128 tokens of one batch item x 256 output features (two
+// heads): warp 0 loads x and w tiles of 64 input channels by TMA into a
+// 4-stage ring, warp 1 issues the MMAs (M = 128, N = 256, K = 16 per
+// instruction) and allocates the 256 tensor-memory columns, warps 2-5 (one
+// thread per token row, lanes by warp & 3) run the epilogue: per head, a
+// first pass over the accumulator for the block maxima, a second for the
+// codes.  The two 64-token blocks of the tile are rows 0-63 (warps 4-5) and
+// 64-127 (warps 2-3).
+#include <cuda_bf16.h>
+
+#include "fp8_codes.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+#include "rope_exact.cuh"
+
+namespace dit {
+namespace {
+
+constexpr int kBM = 128;                   // tokens per tile
+constexpr int kBN = 256;                   // output features per tile (two heads)
+constexpr int kBK = 64;                    // input channels per stage (one 128-byte swizzle row)
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;     // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;     // 32 KB
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kBarEpi = 1;
+
+struct __align__(1024) Smem {
+  uint8_t a[kStages][kABytes];
+  uint8_t b[kStages][kBBytes];
+  uint64_t full[kStages], empty[kStages];
+  uint64_t acc_full;
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort;
+  float block_max[4];                      // per lane quarter of the epilogue warps
+};
+
+struct Params {
+  const float* bias;        // [3 H D] or nullptr
+  const float* cos;         // [N][64] or nullptr
+  const float* sin;
+  uint8_t* codes[3];        // q8, k8, v8: [B][H][N][128]
+  float* scales[3];         // [B][H][ceil(N/64)]
+  __nv_bfloat16* y16[3];    // optional bf16 q, k, v [B][H][N][128] (nullptr: not written)
+  int* status;
+  int N, C, H;
+  int k_steps;
+};
+
+__device__ __forceinline__ void producer(Smem& sm, const Params& p, const CUtensorMap* tm_x, const CUtensorMap* tm_w,
+                                         int n0, int o0, int b, const WaitCtx& wc) {
+  tma_prefetch_desc(tm_x);
+  tma_prefetch_desc(tm_w);
+  int issued = 0;
+  for (int k = 0; k < p.k_steps; ++k) {
+    const int s = k % kStages;
+    const uint32_t ph = (k / kStages) & 1;
+    if (!mbar_wait(&sm.empty[s], ph ^ 1, wc)) break;
+    mbar_arrive_expect_tx(&sm.full[s], kABytes + kBBytes);
+    tma_load_3d(sm.a[s], tm_x, &sm.full[s], k * kBK, n0, b);
+    tma_load_3d(sm.b[s], tm_w, &sm.full[s], k * kBK, o0, 0);
+    issued = k + 1;
+  }
+  if (*wc.abort) {
+    // let the copies already issued land before the CTA exits
+    for (int k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
+      mbar_wait_drain(&sm.full[k % kStages], (k / kStages) & 1, wc);
+  }
+}
+
+__device__ __forceinline__ void mma_issuer(Smem& sm, const Params& p, uint32_t tmem, const WaitCtx& wc) {
+  constexpr uint32_t idesc = instr_desc(1, 1, kBM, kBN, 0, 0);    // bf16 x bf16 -> fp32, both K-major
+  const uint64_t a0 = smem_desc_sw128(smem_u32(sm.a[0]), 16, 1024);
+  const uint64_t b0 = smem_desc_sw128(smem_u32(sm.b[0]), 16, 1024);
+  bool ok = true;
+  for (int k = 0; k < p.k_steps; ++k) {
+    const int s = k % kStages;
+    if (!(ok = mbar_wait(&sm.full[s], (k / kStages) & 1, wc))) break;
+    tc_fence_after();
+    const uint64_t ad = a0 + static_cast<uint32_t>(s) * (kABytes >> 4);
+    const uint64_t bd = b0 + static_cast<uint32_t>(s) * (kBBytes >> 4);
+#pragma unroll
+    for (int kk = 0; kk < kBK / 16; ++kk)   // 16 channels = 32 bytes along the swizzled row
+      mma_ss(tmem, ad + kk * 2, bd + kk * 2, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+    tc_commit(&sm.empty[s]);
+  }
+  if (ok) tc_commit(&sm.acc_full);
+  // every MMA issued above has completed once this arrives
+  tc_commit(&sm.mma_drain);
+  mbar_wait_drain(&sm.mma_drain, 0, wc);
+}
+
+// The 32 accumulator columns at taddr of this thread's row (a warp-collective
+// load: every lane calls it), bias added: y.
+__device__ __forceinline__ void load_y(uint32_t taddr, const Params& p, int o_col, float* y) {
+  uint32_t u[32];
+  tmem_ld32(taddr, u);
+  tmem_ld_wait(u);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(u[e]) + (p.bias != nullptr ? __ldg(p.bias + o_col + e) : 0.f);
+}
+
+// y in place: for q / k each pair rotated with token n's table entries.
+__device__ __forceinline__ void rotate_pairs(const Params& p, int o_col, int n, bool rotate, float* r) {
+  if (rotate) {
+    const int pair0 = (o_col & 127) >> 1;       // first channel pair of the chunk within its head
+    const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(n) * 64 + pair0);
+    const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(n) * 64 + pair0);
+#pragma unroll
+    for (int qd = 0; qd < 4; ++qd) {
+      const float4 cc = __ldg(c4 + qd), ss = __ldg(s4 + qd);
+      const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 8 * qd + 2 * e;
+        const float a = r[i], bb = r[i + 1];
+        r[i] = rot_f64(a, cs[e], bb, -sn[e]);
+        r[i + 1] = rot_f64(a, sn[e], bb, cs[e]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void epilogue(Smem& sm, const Params& p, uint32_t tmem, int n0, int o0, int b, int warp,
+                                         int lane, const WaitCtx& wc) {
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;
+  const int n = n0 + row;
+  const bool valid = n < p.N;
+  const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+  const int nb = (p.N + 63) / 64;
+  const bool ok = warp_wait(&sm.acc_full, 0, wc);
+  tc_fence_after();
+#pragma unroll 1
+  for (int head = 0; head < kBN / 128; ++head) {
+    const int o_head = o0 + head * 128;            // first output feature of the head
+    const int which = o_head / (p.H * 128);        // 0 q, 1 k, 2 v
+    const int h = (o_head / 128) % p.H;
+    const bool rotate = which < 2 && p.cos != nullptr && valid;
+    const uint32_t tcol = tmem + lane_base + head * 128;
+    // pass 1: the row's amax, then the block's (and the optional bf16 y)
+    float amax = 0.f;
+    if (ok) {
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float r[32];
+        load_y(tcol + q * 32, p, o_head + q * 32, r);
+        if (valid && p.y16[which] != nullptr) {
+          // unrotated y, rounded to bf16, in the attention layout
+          uint4* dst = reinterpret_cast<uint4*>(p.y16[which] +
+                                                ((static_cast<size_t>(b) * p.H + h) * p.N + n) * 128 + q * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16x2_rn(r[8 * e], r[8 * e + 1]), pack_bf16x2_rn(r[8 * e + 2], r[8 * e + 3]),
+                                pack_bf16x2_rn(r[8 * e + 4], r[8 * e + 5]), pack_bf16x2_rn(r[8 * e + 6], r[8 * e + 7]));
+        }
+        rotate_pairs(p, o_head + q * 32, n, rotate, r);
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(r[e]));
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) sm.block_max[quarter] = amax;
+    named_bar_sync(kBarEpi, kEpiThreads);
+    const int blk = row >> 6;                      // 64-token block of the tile: quarters 0-1, 2-3
+    const float bmax = fmaxf(sm.block_max[2 * blk], sm.block_max[2 * blk + 1]);
+    named_bar_sync(kBarEpi, kEpiThreads);          // block_max is reused by the next head
+    const float scale = bmax == 0.f ? 1.0f : __fdiv_rn(bmax, 448.0f);
+    if ((row & 63) == 0 && valid)
+      p.scales[which][(static_cast<size_t>(b) * p.H + h) * nb + (n0 >> 6) + blk] = scale;
+    if (!ok) continue;
+    // pass 2: the codes of r / scale (the reciprocal decides when it can);
+    // every lane takes part in the warp-collective loads, valid rows store
+    const bool via_reciprocal = scale >= 1.17549435e-38f && scale <= 8.50705917e+37f;
+    const float rs = __frcp_rn(scale);
+    uint8_t* out = p.codes[which] + ((static_cast<size_t>(b) * p.H + h) * p.N + n) * 128;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      float r[32];
+      load_y(tcol + q * 32, p, o_head + q * 32, r);
+      rotate_pairs(p, o_head + q * 32, n, rotate, r);
+      uint32_t word[8];
+#pragma unroll
+      for (int w4 = 0; w4 < 8; ++w4) {
+        uint32_t wd = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x = r[4 * w4 + e];
+          uint32_t code;
+          if (!via_reciprocal || !e4m3_of_quotient(x, rs, code)) code = e4m3x2(__fdiv_rn(x, scale), 0.f) & 0xFFu;
+          wd |= code << (8 * e);
+        }
+        word[w4] = wd;
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + q * 32);
+        dst[0] = make_uint4(word[0], word[1], word[2], word[3]);
+        dst[1] = make_uint4(word[4], word[5], word[6], word[7]);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    qkv_proj_fp8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                        const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBM;
+  const int o0 = blockIdx.y * kBN;
+  const int b = blockIdx.z;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.mma_drain, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort, p.status, 0u};
+  if (warp == 0) {
+    if (lane == 0) producer(sm, p, &tm_x, &tm_w, n0, o0, b, wc);
+  } else if (warp == 1) {
+    if (lane == 0) mma_issuer(sm, p, tmem, wc);
+  } else {
+    epilogue(sm, p, tmem, n0, o0, b, warp, lane, wc);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kBN);
+}
+
+bool make_map(CUtensorMap* map, const void* base, int inner, int rows, int planes, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2,
+                                 static_cast<cuuint64_t>(inner) * rows * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr) return false;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int launch_qkv_proj_fp8(const QkvProjArgs& a, cudaStream_t s) {
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, a.x, a.C, a.N, a.B, kBM) || !make_map(&mw, a.w, a.C, 3 * a.H * 128, 1, kBN)) return -4;
+  Params p;
+  p.bias = a.bias;
+  p.cos = a.cos;
+  p.sin = a.sin;
+  for (int i = 0; i < 3; ++i) {
+    p.codes[i] = a.codes[i];
+    p.scales[i] = a.scales[i];
+    p.y16[i] = static_cast<__nv_bfloat16*>(a.y16[i]);
+  }
+  p.status = device_status_word();
+  if (p.status == nullptr) return -4;
+  p.N = a.N;
+  p.C = a.C;
+  p.H = a.H;
+  p.k_steps = (a.C + kBK - 1) / kBK;
+  const size_t smem = sizeof(Smem) + 1024;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -4;
+  if (configured_device != dev) {
+    if (cudaFuncSetAttribute(qkv_proj_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -4;
+    configured_device = dev;
+  }
+  const dim3 grid((a.N + kBM - 1) / kBM, 3 * a.H * 128 / kBN, a.B);
+  qkv_proj_fp8_kernel<<<grid, kThreads, smem, s>>>(mx, mw, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+}  // namespace dit

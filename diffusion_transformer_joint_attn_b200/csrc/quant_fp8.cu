@@ -1,6 +1,8 @@
 // FP8 E4M3 block quantisation of Q / K / V for the FP8 attention variant.
 //
-// One CTA per block of 64 tokens x 128 channels of one (b, h).  With rotary
+// A persistent grid of CTAs walks the blocks of 64 tokens x 128 channels of
+// one (b, h), one block per CTA at a time, with the next block's loads in
+// flight while the current one is reduced and encoded.  With rotary
 // tables, each pair is first turned exactly as in fp64 with the fp32 table
 // entries (x c - y s with both products exact, one rounding) and rounded to
 // fp32.  The block's scale is amax / 448 in fp32 (1 for an all-zero block);
@@ -11,6 +13,7 @@
 // a few ulps of an E4M3 rounding midpoint.
 #include <cuda_fp8.h>
 
+#include "fp8_codes.cuh"
 #include "launch.h"
 
 namespace dit {
@@ -20,37 +23,6 @@ constexpr int kBlockTokens = 64;
 constexpr int kThreads = 256;
 constexpr int kChunks = kBlockTokens * 128 / 8;         // 8 channels per chunk
 constexpr int kPerThread = kChunks / kThreads;          // 4
-
-__device__ __forceinline__ float rot_f64(float a, float c, float b, float d) {
-  // a c + b d with exact products, rounded once to fp64, then to fp32
-  const double bd = static_cast<double>(b) * static_cast<double>(d);
-  return static_cast<float>(fma(static_cast<double>(a), static_cast<double>(c), bd));
-}
-
-// E4M3 codes of lo (low byte) and hi (high byte), nearest even, saturating.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// E4M3 code of the correctly rounded fp32 quotient x / scale from
-// r = 1 / scale rounded to nearest (scale and r normal); false if undecided.
-// x * r is within 3 fp32 ulps of that quotient: r and the product are each
-// rounded once, with relative error at most 2^-24.  Rounding to E4M3 is
-// monotonic, so when the fp32 values 8 ulps below and above x * r (the lower
-// magnitude clamped at 0) have one code, the quotient has it too.  They
-// differ when the quotient lies within a few ulps of an E4M3 rounding
-// midpoint (or is not finite); the caller then divides.
-__device__ __forceinline__ bool e4m3_of_quotient(float x, float r, uint32_t& code) {
-  const uint32_t u = __float_as_uint(x * r);
-  const uint32_t mag = u & 0x7FFFFFFFu;
-  const float below = __uint_as_float((u & 0x80000000u) | (max(mag, 8u) - 8u));
-  const float above = __uint_as_float(u + 8u);
-  const uint32_t two = e4m3x2(below, above);
-  code = two & 0xFFu;
-  return ((two ^ (two >> 8)) & 0xFFu) == 0u;
-}
 
 // Element e (0..7) of a chunk held as fp32 values (rotated) or as the raw
 // bf16 words (unrotated: half the registers, so more CTAs stay resident).
@@ -69,14 +41,26 @@ struct Chunk<false> {
   }
 };
 
+// The raw 16-byte chunks this thread loads of block `blk` (zeros past N).
+__device__ __forceinline__ void load_block(const uint4* __restrict__ x, long long blk, int N, int blocks_per_bh,
+                                           uint4* raw) {
+  const long long bh = blk / blocks_per_bh;
+  const int n0 = static_cast<int>(blk % blocks_per_bh) * kBlockTokens;
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int c = threadIdx.x + u * kThreads;
+    const int n = n0 + (c >> 4);               // 16 chunks per token row
+    raw[u] = n < N ? __ldg(x + (bh * N + n) * 16 + (c & 15)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 template <bool kRotate>
-__device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, const float* __restrict__ tc,
+__device__ __forceinline__ void quantize_block(const uint4* raw, const float* __restrict__ tc,
                                                const float* __restrict__ ts, uint2* __restrict__ codes,
-                                               float* __restrict__ scales, int N, int blocks_per_bh) {
-  __shared__ float warp_max[kThreads / 32];
-  const int bh = blockIdx.x / blocks_per_bh;
-  const int blk = blockIdx.x % blocks_per_bh;
-  const int n0 = blk * kBlockTokens;
+                                               float* __restrict__ scales, int N, int blocks_per_bh, long long blk,
+                                               float* warp_max) {
+  const long long bh = blk / blocks_per_bh;
+  const int n0 = static_cast<int>(blk % blocks_per_bh) * kBlockTokens;
   Chunk<kRotate> ch[kPerThread];
   float amax = 0.f;
 #pragma unroll
@@ -85,8 +69,7 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
     const int r = c >> 4;                      // 16 chunks per token row
     const int n = n0 + r;
     if (n < N) {
-      const long long idx = (static_cast<long long>(bh) * N + n) * 16 + (c & 15);
-      const uint4 w = __ldg(x + idx);
+      const uint4 w = raw[u];
       if constexpr (kRotate) {
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
         // the four pairs of this chunk: table entries n * 64 + (c & 15) * 4 + 0..3
@@ -114,7 +97,7 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
 #pragma unroll
   for (int w = 1; w < kThreads / 32; ++w) bmax = fmaxf(bmax, warp_max[w]);
   const float scale = bmax == 0.f ? 1.0f : __fdiv_rn(bmax, 448.0f);
-  if (threadIdx.x == 0) scales[blockIdx.x] = scale;
+  if (threadIdx.x == 0) scales[blk] = scale;
   // the reciprocal path needs scale and 1 / scale normal: scale in [2^-126, 2^126]
   const bool via_reciprocal = scale >= 1.17549435e-38f && scale <= 8.50705917e+37f;
   const float r = __frcp_rn(scale);
@@ -140,34 +123,64 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
         }
       }
     }
-    codes[(static_cast<long long>(bh) * N + n) * 16 + (c & 15)] = make_uint2(word[0], word[1]);
+    codes[(bh * N + n) * 16 + (c & 15)] = make_uint2(word[0], word[1]);
   }
 }
 
-// q, k (rotated): 64 registers, 4 CTAs per SM.  v: the raw words take fewer
-// registers, and 5 CTAs per SM keep more loads in flight.
+// Blocks blockIdx.x, blockIdx.x + gridDim.x, ...: the loads of the next
+// block are issued before the current one is reduced and encoded.  The block
+// maxima go through shared memory in two alternating sets, so one barrier
+// per block suffices.
+template <bool kRotate>
+__device__ __forceinline__ void quantize_blocks(const uint4* __restrict__ x, const float* __restrict__ tc,
+                                                const float* __restrict__ ts, uint2* __restrict__ codes,
+                                                float* __restrict__ scales, int N, int blocks_per_bh,
+                                                long long blocks) {
+  __shared__ float warp_max[2][kThreads / 32];
+  uint4 cur[kPerThread], nxt[kPerThread];
+  long long blk = blockIdx.x;
+  if (blk < blocks) load_block(x, blk, N, blocks_per_bh, cur);
+  for (int i = 0; blk < blocks; ++i, blk += gridDim.x) {
+    if (blk + gridDim.x < blocks) load_block(x, blk + gridDim.x, N, blocks_per_bh, nxt);
+    quantize_block<kRotate>(cur, tc, ts, codes, scales, N, blocks_per_bh, blk, warp_max[i & 1]);
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) cur[u] = nxt[u];
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
                                                             const float* __restrict__ ts, uint2* __restrict__ codes,
-                                                            float* __restrict__ scales, int N, int blocks_per_bh) {
-  quantize_block<true>(x, tc, ts, codes, scales, N, blocks_per_bh);
+                                                            float* __restrict__ scales, int N, int blocks_per_bh,
+                                                            long long blocks) {
+  quantize_blocks<true>(x, tc, ts, codes, scales, N, blocks_per_bh, blocks);
 }
-__global__ void __launch_bounds__(kThreads, 5)
+__global__ void __launch_bounds__(kThreads)
     quantize_unrotated_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes, float* __restrict__ scales, int N,
-                              int blocks_per_bh) {
-  quantize_block<false>(x, nullptr, nullptr, codes, scales, N, blocks_per_bh);
+                              int blocks_per_bh, long long blocks) {
+  quantize_blocks<false>(x, nullptr, nullptr, codes, scales, N, blocks_per_bh, blocks);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_fp8(const QuantFp8Args& a, cudaStream_t s) {
   const int blocks_per_bh = (a.N + kBlockTokens - 1) / kBlockTokens;
-  const long long grid = static_cast<long long>(a.B) * a.H * blocks_per_bh;
+  const long long blocks = static_cast<long long>(a.B) * a.H * blocks_per_bh;
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // a persistent grid: exactly the CTAs that are resident at once (a CTA
+  // beyond that would start its share of the blocks only in a second wave)
+  cudaError_t r = a.cos != nullptr
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel, kThreads, 0)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_unrotated_kernel, kThreads, 0);
+  if (r != cudaSuccess) return r;
+  const long long cap = static_cast<long long>(sms) * (per_sm > 0 ? per_sm : 1);
+  const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
   if (a.cos != nullptr)
-    quantize_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
-        static_cast<const uint4*>(a.x), a.cos, a.sin, static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh);
+    quantize_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(a.x), a.cos, a.sin,
+                                              static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh, blocks);
   else
-    quantize_unrotated_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
-        static_cast<const uint4*>(a.x), static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh);
+    quantize_unrotated_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(a.x), static_cast<uint2*>(a.codes),
+                                                        a.scale, a.N, blocks_per_bh, blocks);
   return cudaGetLastError();
 }
 

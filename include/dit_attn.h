@@ -368,6 +368,47 @@ int dit_attn_forward_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8
                          int N_txt, int N_img, int D, int dtype, dit_stream_t stream);
 
 /*
+ * dit_qkv_project_fp8 — the QKV projection of the joint token sequence with
+ * the FP8 operands of dit_attn_forward_fp8 made in the GEMM's epilogue
+ * (the pages list GEMMs with epilogue fusion among the optimisations of
+ * FLUX 3 Klein on B200: bpdata.com "FLUX 3 Image Klein optimalizálása",
+ * sections on what the optimisation includes and on the detailed steps):
+ *
+ *     y[b][n][o] = sum_c x[b][n][c] w[o][c] (+ bias[o]),   o = s*H*D + h*D + d
+ *
+ * for s = 0, 1, 2 (q, k, v), accumulated in fp32 on the tensor cores, then,
+ * per (s, b, h) without writing y to memory: q and k rotated exactly as by
+ * dit_attn_quantize_fp8 (each pair turned in fp64 from the fp32 y and the fp32
+ * table entries, rounded to fp32), and every block of 64 tokens x D channels
+ * quantised as by dit_attn_quantize_fp8 (scale = amax / 448 in fp32, 1 for an
+ * all-zero block; codes = E4M3 of y / scale, nearest even, saturating).
+ *
+ *   x         device bf16 [B][N][C]: hidden states of the joint sequence.
+ *   w         device bf16 [3 H D][C]: the projection weight (rows: q heads,
+ *             then k heads, then v heads; row-major like a linear layer).
+ *   bias      device fp32 [3 H D] or NULL.
+ *   rope_cos, rope_sin
+ *             device fp32 [N][D/2] (dit_rope_table_build) or both NULL.
+ *   q8, k8, v8
+ *             device uint8 [B][H][N][D], written: E4M3 codes.
+ *   q_scale, k_scale, v_scale
+ *             device fp32 [B][H][ceil(N/64)], written.
+ *   q16, k16, v16
+ *             device bf16 [B][H][N][D] or NULL: the unrotated projection
+ *             rounded to bf16 (the inputs of the BF16 path), written if given.
+ *   B, N      >= 1.  C >= 1 with C % 8 == 0.  H >= 1 and even (256 output
+ *             features per tile).  D must be 128.
+ * Pointers 16-byte aligned except bias and the scales (4-byte).  Because the
+ * sums are formed in fp32 in the tensor cores' order, a code can differ by
+ * one step from the code of the exact projection where y / scale lies
+ * within the accumulation error of a rounding midpoint.
+ */
+int dit_qkv_project_fp8(const void* x, const void* w, const float* bias, const float* rope_cos,
+                        const float* rope_sin, uint8_t* q8, uint8_t* k8, uint8_t* v8, float* q_scale, float* k_scale,
+                        float* v_scale, void* q16, void* k16, void* v16, int B, int N, int C, int H, int D,
+                        dit_stream_t stream);
+
+/*
  * dit_attn_merge — combine R partial results of the same queries over
  * disjoint key sets into the result over their union (context parallelism:
  * wavespeed.ai "Beschleunigung der FLUX.1-dev Bildgenerierung", section on

@@ -115,6 +115,29 @@ def test_key_set_forward_argument_errors(lib):
     assert call(cos=0x50000, sin=0x60000, dtype=dit.DIT_QK_SPLIT) == dit.DIT_ERR_INVALID_ARG   # v fp16 required
 
 
+def test_projection_argument_errors(lib):
+    f = lib.dit_qkv_project_fp8
+    ok = dict(x=0x10000, w=0x20000, bias=None, c=None, s=None, q8=0x30000, k8=0x40000, v8=0x50000, qs=0x60000,
+              ks=0x70000, vs=0x80000, q16=None, k16=None, v16=None, B=1, N=64, C=128, H=2, D=128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["x"], a["w"], a["bias"], a["c"], a["s"], a["q8"], a["k8"], a["v8"], a["qs"], a["ks"], a["vs"],
+                 a["q16"], a["k16"], a["v16"], a["B"], a["N"], a["C"], a["H"], a["D"], None)
+    assert call(x=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(vs=None) == dit.DIT_ERR_INVALID_ARG
+    assert call(c=0x90000) == dit.DIT_ERR_INVALID_ARG          # sin missing
+    assert call(N=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(C=0) == dit.DIT_ERR_INVALID_ARG
+    assert call(D=64) == dit.DIT_ERR_UNSUPPORTED
+    assert call(H=3) == dit.DIT_ERR_UNSUPPORTED                 # two heads per tile
+    assert call(C=100) == dit.DIT_ERR_UNSUPPORTED               # rows of x and w 16-byte aligned
+    assert call(x=0x10008) == dit.DIT_ERR_MISALIGNED
+    assert call(q8=0x30004) == dit.DIT_ERR_MISALIGNED
+    assert call(bias=0x90002) == dit.DIT_ERR_MISALIGNED
+    assert call(k16=0xA0008) == dit.DIT_ERR_MISALIGNED
+
+
 def test_sparse_forward_argument_errors(lib):
     f = lib.dit_attn_forward_sparse
 

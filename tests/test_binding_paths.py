@@ -105,6 +105,21 @@ def test_split_and_key_set_wrappers():
                                 dit.DIT_K_ROTATED | dit.DIT_V_F16 | dit.DIT_OUT_F32, stream=0)
 
 
+def test_projection_wrapper():
+    C, H = 256, 2
+    x, w = OnGpu((B, N, C), bf16), OnGpu((3 * H * 128, C), bf16)
+    codes = [OnGpu((B, H, N, D), u8) for _ in range(3)]
+    scales = [OnGpu((B, H, (N + 63) // 64), f32) for _ in range(3)]
+    y16 = [OnGpu((B, H, N, D), bf16) for _ in range(3)]
+    c, s = OnGpu((N, 64), f32), OnGpu((N, 64), f32)
+    fails_at_cuda(lambda: dit.dit_qkv_project_fp8(x, w, OnGpu((3 * H * 128,), f32), c, s, *codes, *scales, *y16,
+                                                  stream=0))
+    fails_at_cuda(lambda: dit.dit_qkv_project_fp8(x, w, None, None, None, *codes, *scales, stream=0))
+    with pytest.raises(ValueError, match="scales"):
+        dit.dit_qkv_project_fp8(x, w, None, None, None, *codes, scales[0], scales[1], OnGpu((B, H, 2), f32),
+                                stream=0)
+
+
 def test_fp8_wrappers():
     x = OnGpu((B, H, N, D), bf16)
     codes, scale = OnGpu((B, H, N, D), u8), OnGpu((B, H, 1), f32)

@@ -265,3 +265,46 @@ def test_bounded_wait_times_out_reports_and_leaves_the_context_usable():
     out32, lse32 = run_gpu(w, out_f32=True, inputs=inputs)
     O_op, L_op = oracle_rows(w, q, k, v, rows, operands="bf16")
     check(out32, lse32, rows, O_op, L_op, "after a timed-out wait")
+
+
+def test_step_replays_in_a_cuda_graph():
+    """The hot path makes stream-ordered launches only (no host sync, no
+    allocation), so a step - rotary table, K/V operand pass, forward - can
+    be captured in a CUDA graph once a first call outside any capture has set
+    the kernels up; replays equal direct calls bit for bit, also after the
+    inputs change in place."""
+    w = W.WORKLOADS["t2i_512px"]
+    _, _, _, qd, kd, vd = device_inputs(w)
+    pos = torch.from_numpy(W.positions(w)).cuda()
+    c = torch.empty((w.N, 64), dtype=torch.float32, device="cuda")
+    s = torch.empty_like(c)
+    kr = torch.empty_like(kd)
+    v16 = torch.empty(vd.shape, dtype=torch.float16, device="cuda")
+    out = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    flags = dit.DIT_BF16 | dit.DIT_K_ROTATED | dit.DIT_V_F16
+
+    def step():
+        dit.dit_rope_table_build(pos, (16, 56, 56), 10000.0, c, s)
+        dit.dit_attn_prepare_kv(kd, vd, c, s, kr, v16)
+        dit.dit_attn_forward(qd, kr, v16, c, s, out, lse, w.n_txt, w.n_img, flags)
+
+    step()                                   # first call outside any capture
+    torch.cuda.synchronize()
+    ref, ref_lse = out.clone(), lse.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+    qd.copy_(torch.flip(qd, dims=[2]))       # new inputs in the captured buffers
+    graph.replay()
+    torch.cuda.synchronize()
+    graphed, graphed_lse = out.clone(), lse.clone()
+    step()
+    torch.cuda.synchronize()
+    assert torch.equal(graphed, out) and torch.equal(graphed_lse, lse)
+    assert not torch.equal(graphed, ref)
+    assert dit.dit_attn_get_status() == dit.DIT_OK

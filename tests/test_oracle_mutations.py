@@ -9,7 +9,8 @@ import pytest
 
 import test_oracle_attention as TA
 import test_oracle_formats as TF
-from oracle import attention, formats, fp8, merge, rope
+import test_oracle_projection as TP
+from oracle import attention, formats, fp8, merge, projection, rope
 
 
 # ---------------------------------------------------------------- planted mistakes
@@ -97,7 +98,20 @@ def _fp32_chopped(x):
     return x.astype(np.float32).astype(np.float64) * (1.0 - 2.0 ** -24)
 
 
-_ORIG = {"round_fp16": formats.round_fp16, "frequencies": rope.frequencies, "attention_rows": attention.attention_rows, "merge": merge.merge,
+def _projection_head_major(x, w, bias=None, H=24, D=128):
+    y = np.einsum("bnc,oc->bno", attention.to_f64(x), attention.to_f64(w))
+    if bias is not None:
+        y = y + attention.to_f64(bias)[None, None, :]
+    B, N, _ = y.shape
+    y = y.reshape(B, N, H, 3, D).transpose(3, 0, 2, 1, 4)            # features read as (h, s, d)
+    return y[0], y[1], y[2]
+
+
+def _projection_without_bias(x, w, bias=None, H=24, D=128):
+    return _ORIG["project"](x, w, None, H=H, D=D)
+
+
+_ORIG = {"project": projection.project, "round_fp16": formats.round_fp16, "frequencies": rope.frequencies, "attention_rows": attention.attention_rows, "merge": merge.merge,
          "block_scales": fp8.block_scales}
 
 # pins, as callables without arguments
@@ -108,6 +122,7 @@ P_ROPE = [TA.test_rope_rotation_direction, TA.test_rope_relative_position,
 P_ATTN = [TA.test_rows_sum_to_one, TA.test_zero_query_gives_column_mean_and_log_n,
           TA.test_dominant_key_returns_its_value_row, lambda: TA.test_matches_library_sdpa_without_rope(64)]
 P_MERGE = [TA.test_merge_of_key_slices_equals_full_attention, TA.test_merge_weights_follow_the_softmax_of_the_lses]
+P_PROJ = [TP.test_project_matches_exact_rational_sums, TP.test_project_regroups_features_into_q_k_v_heads]
 P_SPLIT = [TF.test_split_fp16_terms, TF.test_round_fp32_matches_library_cast_and_ties_to_even]
 P_FP8 = [TF.test_block_quantisation_properties, TF.test_e4m3_midpoints_round_to_even_and_saturate,
          TF.test_e4m3_encode_matches_library_cast, TF.test_e4m3_landmark_codes]
@@ -126,6 +141,8 @@ MUTATIONS = [
     ("split remainder not rounded", formats, "split_fp16", _split_remainder_unrounded, P_SPLIT),
     ("split hi chopped", formats, "split_fp16", _split_truncated, P_SPLIT),
     ("fp32 rounding biased", formats, "round_fp32", _fp32_chopped, P_SPLIT),
+    ("projection features read head-major", projection, "project", _projection_head_major, P_PROJ),
+    ("projection bias dropped", projection, "project", _projection_without_bias, P_PROJ),
 ]
 
 
@@ -142,5 +159,5 @@ def test_planted_mistake_fails_a_pin(name, module, attr, bad, pins, monkeypatch)
 
 
 def test_pins_pass_on_the_unmodified_oracle():
-    for pin in P_BRUTE + P_ROPE + P_ATTN + P_MERGE + P_FP8 + P_SPLIT:
+    for pin in P_BRUTE + P_ROPE + P_ATTN + P_MERGE + P_FP8 + P_SPLIT + P_PROJ:
         pin()
