@@ -13,7 +13,10 @@
 // optionally also the unrotated y rounded to bf16 in the attention layout.
 //
 // One CTA per tile of 128 tokens of one batch item x 256 output features (two
-// heads): warp 0 loads x and w tiles of 64 input channels by TMA into a
+// heads; pairs of CTAs with four heads further down).  blockIdx.x runs over
+// the feature tiles, so the CTAs resident at once share their token rows of
+// x and sweep the whole weight, which (57 MB at the FLUX width) stays in L2,
+// while x is read from HBM about once.  Warp 0 loads x and w tiles of 64 input channels by TMA into a
 // 4-stage ring, warp 1 issues the MMAs (M = 128, N = 256, K = 16 per
 // instruction) and allocates the 256 tensor-memory columns, warps 2-5 (one
 // thread per token row, lanes by warp & 3) run the epilogue: per head, a
@@ -137,7 +140,10 @@ __device__ __forceinline__ void rotate_pairs(const Params& p, int o_col, int n, 
   }
 }
 
-__device__ __forceinline__ void epilogue(Smem& sm, const Params& p, uint32_t tmem, int n0, int o0, int b, int warp,
+// kHeads heads of 128 accumulator columns each, for the 128 token rows of
+// this CTA starting at token n0; sm supplies acc_full and block_max.
+template <int kHeads, typename SmemT>
+__device__ __forceinline__ void epilogue(SmemT& sm, const Params& p, uint32_t tmem, int n0, int o0, int b, int warp,
                                          int lane, const WaitCtx& wc) {
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
@@ -148,7 +154,7 @@ __device__ __forceinline__ void epilogue(Smem& sm, const Params& p, uint32_t tme
   const bool ok = warp_wait(&sm.acc_full, 0, wc);
   tc_fence_after();
 #pragma unroll 1
-  for (int head = 0; head < kBN / 128; ++head) {
+  for (int head = 0; head < kHeads; ++head) {
     const int o_head = o0 + head * 128;            // first output feature of the head
     const int which = o_head / (p.H * 128);        // 0 q, 1 k, 2 v
     const int h = (o_head / 128) % p.H;
@@ -227,8 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBM;
-  const int o0 = blockIdx.y * kBN;
+  const int n0 = blockIdx.y * kBM;
+  const int o0 = blockIdx.x * kBN;
   const int b = blockIdx.z;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -254,13 +260,149 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) mma_issuer(sm, p, tmem, wc);
   } else {
-    epilogue(sm, p, tmem, n0, o0, b, warp, lane, wc);
+    epilogue<kBN / 128>(sm, p, tmem, n0, o0, b, warp, lane, wc);
   }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kBN);
+}
+
+// ---------------------------------------------------------------- CTA pairs
+// When H is a multiple of 4: a cluster of two CTAs computes 256 tokens (128
+// per CTA) x 512 output features (four heads) with pair MMAs (M = 256,
+// N = 256, two per 16 input channels, into tensor-memory columns 0-255 and
+// 256-511).  Each CTA loads its own 128 token rows of x and, for each of the
+// two MMAs, its half (128 features) of the weight rows; the pair MMA reads
+// both CTAs' halves.  Per 64 input channels a CTA loads 48 KB for 2 x 128 x
+// 512 x 64 FLOP, 2/3 of the bytes per FLOP of the one-CTA tile (L2 to SMEM
+// traffic is what bounds that tile).  The epilogue of each CTA is the one
+// above, for four heads.
+constexpr int kPairBN = 512;
+constexpr int kPairBHalf = 128 * kBK * 2;   // 16 KB: 128 weight rows of one MMA
+constexpr int kPairStageBytes = kABytes + 2 * kPairBHalf;
+
+struct __align__(1024) PairSmem {
+  uint8_t a[kStages][kABytes];
+  uint8_t b[kStages][2][kPairBHalf];
+  uint64_t full[kStages], empty[kStages];   // full: the even CTA's counts both CTAs' bytes
+  uint64_t acc_full;
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort;
+  float block_max[4];
+};
+
+__device__ __forceinline__ uint32_t cl_addr(const void* p, uint32_t rank) { return mapa_shared(smem_u32(p), rank); }
+
+__device__ __forceinline__ void pair_producer(PairSmem& sm, const Params& p, const CUtensorMap* tm_x,
+                                              const CUtensorMap* tm_w, int n0, int o0, int b, uint32_t rank,
+                                              const WaitCtx& wc) {
+  tma_prefetch_desc(tm_x);
+  tma_prefetch_desc(tm_w);
+  int issued = 0;
+  for (int k = 0; k < p.k_steps; ++k) {
+    const int s = k % kStages;
+    const uint32_t ph = (k / kStages) & 1;
+    if (!mbar_wait(&sm.empty[s], ph ^ 1, wc)) break;
+    if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * kPairStageBytes);
+    const uint32_t bar = cl_addr(&sm.full[s], 0);
+    tma_load_3d_pair(sm.a[s], tm_x, bar, k * kBK, n0, b);
+    for (int m = 0; m < 2; ++m)
+      tma_load_3d_pair(sm.b[s][m], tm_w, bar, k * kBK, o0 + 256 * m + 128 * static_cast<int>(rank), 0);
+    issued = k + 1;
+  }
+  if (*wc.abort) {
+    // let the copies already issued land before the pair exits: the even CTA
+    // counts both CTAs' bytes; the odd CTA waits out a few microseconds
+    if (rank == 0) {
+      for (int k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
+        mbar_wait_drain(&sm.full[k % kStages], (k / kStages) & 1, wc);
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 20000) {
+      }
+    }
+  }
+}
+
+// Even CTA only: completions are signalled to the barrier of the same name in
+// both CTAs.
+__device__ __forceinline__ void pair_mma_issuer(PairSmem& sm, const Params& p, uint32_t tmem, const WaitCtx& wc) {
+  constexpr uint32_t idesc = instr_desc(1, 1, 256, 256, 0, 0);    // bf16 x bf16 -> fp32, both K-major
+  const uint64_t a0 = smem_desc_sw128(smem_u32(sm.a[0]), 16, 1024);
+  const uint64_t b0 = smem_desc_sw128(smem_u32(sm.b[0][0]), 16, 1024);
+  bool ok = true;
+  for (int k = 0; k < p.k_steps; ++k) {
+    const int s = k % kStages;
+    if (!(ok = mbar_wait(&sm.full[s], (k / kStages) & 1, wc))) break;
+    tc_fence_after();
+    const uint64_t ad = a0 + static_cast<uint32_t>(s) * (kABytes >> 4);
+    const uint64_t bd = b0 + static_cast<uint32_t>(s) * ((2 * kPairBHalf) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < kBK / 16; ++kk) {
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+        mma_ss_pair(tmem + 256 * m, ad + kk * 2, bd + m * (kPairBHalf >> 4) + kk * 2, idesc,
+                    (k > 0 || kk > 0) ? 1u : 0u);
+    }
+    tc_commit_pair(cl_addr(&sm.empty[s], 0));
+    tc_commit_pair(cl_addr(&sm.empty[s], 1));
+  }
+  if (ok) {
+    tc_commit_pair(cl_addr(&sm.acc_full, 0));
+    tc_commit_pair(cl_addr(&sm.acc_full, 1));
+  }
+  // every MMA issued above has completed once this arrives
+  tc_commit_pair(cl_addr(&sm.mma_drain, 0));
+  mbar_wait_drain(&sm.mma_drain, 0, wc);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    qkv_proj_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                         const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  PairSmem& sm = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  // clusters are two CTAs along x: blockIdx.x = 2 x (512-feature tile) + rank, so that the
+  // feature tiles of one token tile run next to each other and the weight stays in L2
+  const int n0 = blockIdx.y * 2 * kBM + kBM * static_cast<int>(rank);   // this CTA's first token
+  const int o0 = (blockIdx.x >> 1) * kPairBN;
+  const int b = blockIdx.z;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.mma_drain, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm.tmem_base, kPairBN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();          // both CTAs' barriers initialised, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort, p.status, cl_addr(&sm.abort, rank ^ 1u)};
+  if (warp == 0) {
+    if (lane == 0) pair_producer(sm, p, &tm_x, &tm_w, n0, o0, b, rank, wc);
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) pair_mma_issuer(sm, p, tmem, wc);
+  } else {
+    epilogue<kPairBN / 128>(sm, p, tmem, n0, o0, b, warp, lane, wc);
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();          // no CTA leaves while its peer may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kPairBN);
 }
 
 bool make_map(CUtensorMap* map, const void* base, int inner, int rows, int planes, int box_rows) {
@@ -280,8 +422,10 @@ bool make_map(CUtensorMap* map, const void* base, int inner, int rows, int plane
 }  // namespace
 
 int launch_qkv_proj_fp8(const QkvProjArgs& a, cudaStream_t s) {
+  const bool pair = a.H % 4 == 0;          // 512 output features per cluster
   CUtensorMap mx, mw;
-  if (!make_map(&mx, a.x, a.C, a.N, a.B, kBM) || !make_map(&mw, a.w, a.C, 3 * a.H * 128, 1, kBN)) return -4;
+  if (!make_map(&mx, a.x, a.C, a.N, a.B, kBM) || !make_map(&mw, a.w, a.C, 3 * a.H * 128, 1, pair ? 128 : kBN))
+    return -4;
   Params p;
   p.bias = a.bias;
   p.cos = a.cos;
@@ -297,19 +441,36 @@ int launch_qkv_proj_fp8(const QkvProjArgs& a, cudaStream_t s) {
   p.C = a.C;
   p.H = a.H;
   p.k_steps = (a.C + kBK - 1) / kBK;
-  const size_t smem = sizeof(Smem) + 1024;
+  const size_t smem = sizeof(Smem) + 1024, smem_pair = sizeof(PairSmem) + 1024;
   static thread_local int configured_device = -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -4;
   if (configured_device != dev) {
     if (cudaFuncSetAttribute(qkv_proj_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(qkv_proj_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_pair)) != cudaSuccess)
       return -4;
     configured_device = dev;
   }
-  const dim3 grid((a.N + kBM - 1) / kBM, 3 * a.H * 128 / kBN, a.B);
-  qkv_proj_fp8_kernel<<<grid, kThreads, smem, s>>>(mx, mw, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  if (!pair) {
+    const dim3 grid(3 * a.H * 128 / kBN, (a.N + kBM - 1) / kBM, a.B);
+    qkv_proj_fp8_kernel<<<grid, kThreads, smem, s>>>(mx, mw, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (3 * a.H * 128 / kPairBN), (a.N + 2 * kBM - 1) / (2 * kBM), a.B);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_pair;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qkv_proj_pair_kernel, mx, mw, p) == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace dit

@@ -1,8 +1,6 @@
 // FP8 E4M3 block quantisation of Q / K / V for the FP8 attention variant.
 //
-// A persistent grid of CTAs walks the blocks of 64 tokens x 128 channels of
-// one (b, h), one block per CTA at a time, with the next block's loads in
-// flight while the current one is reduced and encoded.  With rotary
+// One CTA per block of 64 tokens x 128 channels of one (b, h).  With rotary
 // tables, each pair is first turned exactly as in fp64 with the fp32 table
 // entries (x c - y s with both products exact, one rounding) and rounded to
 // fp32.  The block's scale is amax / 448 in fp32 (1 for an all-zero block);
@@ -41,26 +39,14 @@ struct Chunk<false> {
   }
 };
 
-// The raw 16-byte chunks this thread loads of block `blk` (zeros past N).
-__device__ __forceinline__ void load_block(const uint4* __restrict__ x, long long blk, int N, int blocks_per_bh,
-                                           uint4* raw) {
-  const long long bh = blk / blocks_per_bh;
-  const int n0 = static_cast<int>(blk % blocks_per_bh) * kBlockTokens;
-#pragma unroll
-  for (int u = 0; u < kPerThread; ++u) {
-    const int c = threadIdx.x + u * kThreads;
-    const int n = n0 + (c >> 4);               // 16 chunks per token row
-    raw[u] = n < N ? __ldg(x + (bh * N + n) * 16 + (c & 15)) : make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
 template <bool kRotate>
-__device__ __forceinline__ void quantize_block(const uint4* raw, const float* __restrict__ tc,
+__device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, const float* __restrict__ tc,
                                                const float* __restrict__ ts, uint2* __restrict__ codes,
-                                               float* __restrict__ scales, int N, int blocks_per_bh, long long blk,
-                                               float* warp_max) {
-  const long long bh = blk / blocks_per_bh;
-  const int n0 = static_cast<int>(blk % blocks_per_bh) * kBlockTokens;
+                                               float* __restrict__ scales, int N, int blocks_per_bh) {
+  __shared__ float warp_max[kThreads / 32];
+  const int bh = blockIdx.x / blocks_per_bh;
+  const int blk = blockIdx.x % blocks_per_bh;
+  const int n0 = blk * kBlockTokens;
   Chunk<kRotate> ch[kPerThread];
   float amax = 0.f;
 #pragma unroll
@@ -69,7 +55,8 @@ __device__ __forceinline__ void quantize_block(const uint4* raw, const float* __
     const int r = c >> 4;                      // 16 chunks per token row
     const int n = n0 + r;
     if (n < N) {
-      const uint4 w = raw[u];
+      const long long idx = (static_cast<long long>(bh) * N + n) * 16 + (c & 15);
+      const uint4 w = __ldg(x + idx);
       if constexpr (kRotate) {
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
         // the four pairs of this chunk: table entries n * 64 + (c & 15) * 4 + 0..3
@@ -97,7 +84,7 @@ __device__ __forceinline__ void quantize_block(const uint4* raw, const float* __
 #pragma unroll
   for (int w = 1; w < kThreads / 32; ++w) bmax = fmaxf(bmax, warp_max[w]);
   const float scale = bmax == 0.f ? 1.0f : __fdiv_rn(bmax, 448.0f);
-  if (threadIdx.x == 0) scales[blk] = scale;
+  if (threadIdx.x == 0) scales[blockIdx.x] = scale;
   // the reciprocal path needs scale and 1 / scale normal: scale in [2^-126, 2^126]
   const bool via_reciprocal = scale >= 1.17549435e-38f && scale <= 8.50705917e+37f;
   const float r = __frcp_rn(scale);
@@ -123,64 +110,34 @@ __device__ __forceinline__ void quantize_block(const uint4* raw, const float* __
         }
       }
     }
-    codes[(bh * N + n) * 16 + (c & 15)] = make_uint2(word[0], word[1]);
+    codes[(static_cast<long long>(bh) * N + n) * 16 + (c & 15)] = make_uint2(word[0], word[1]);
   }
 }
 
-// Blocks blockIdx.x, blockIdx.x + gridDim.x, ...: the loads of the next
-// block are issued before the current one is reduced and encoded.  The block
-// maxima go through shared memory in two alternating sets, so one barrier
-// per block suffices.
-template <bool kRotate>
-__device__ __forceinline__ void quantize_blocks(const uint4* __restrict__ x, const float* __restrict__ tc,
-                                                const float* __restrict__ ts, uint2* __restrict__ codes,
-                                                float* __restrict__ scales, int N, int blocks_per_bh,
-                                                long long blocks) {
-  __shared__ float warp_max[2][kThreads / 32];
-  uint4 cur[kPerThread], nxt[kPerThread];
-  long long blk = blockIdx.x;
-  if (blk < blocks) load_block(x, blk, N, blocks_per_bh, cur);
-  for (int i = 0; blk < blocks; ++i, blk += gridDim.x) {
-    if (blk + gridDim.x < blocks) load_block(x, blk + gridDim.x, N, blocks_per_bh, nxt);
-    quantize_block<kRotate>(cur, tc, ts, codes, scales, N, blocks_per_bh, blk, warp_max[i & 1]);
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) cur[u] = nxt[u];
-  }
-}
-
+// q, k (rotated): 64 registers, 4 CTAs per SM.  v: the raw words take fewer
+// registers, and 5 CTAs per SM keep more loads in flight.
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
                                                             const float* __restrict__ ts, uint2* __restrict__ codes,
-                                                            float* __restrict__ scales, int N, int blocks_per_bh,
-                                                            long long blocks) {
-  quantize_blocks<true>(x, tc, ts, codes, scales, N, blocks_per_bh, blocks);
+                                                            float* __restrict__ scales, int N, int blocks_per_bh) {
+  quantize_block<true>(x, tc, ts, codes, scales, N, blocks_per_bh);
 }
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 5)
     quantize_unrotated_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes, float* __restrict__ scales, int N,
-                              int blocks_per_bh, long long blocks) {
-  quantize_blocks<false>(x, nullptr, nullptr, codes, scales, N, blocks_per_bh, blocks);
+                              int blocks_per_bh) {
+  quantize_block<false>(x, nullptr, nullptr, codes, scales, N, blocks_per_bh);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_fp8(const QuantFp8Args& a, cudaStream_t s) {
   const int blocks_per_bh = (a.N + kBlockTokens - 1) / kBlockTokens;
-  const long long blocks = static_cast<long long>(a.B) * a.H * blocks_per_bh;
-  int dev = 0, sms = 148, per_sm = 1;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // a persistent grid: exactly the CTAs that are resident at once (a CTA
-  // beyond that would start its share of the blocks only in a second wave)
-  cudaError_t r = a.cos != nullptr
-                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel, kThreads, 0)
-                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_unrotated_kernel, kThreads, 0);
-  if (r != cudaSuccess) return r;
-  const long long cap = static_cast<long long>(sms) * (per_sm > 0 ? per_sm : 1);
-  const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
+  const long long grid = static_cast<long long>(a.B) * a.H * blocks_per_bh;
   if (a.cos != nullptr)
-    quantize_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(a.x), a.cos, a.sin,
-                                              static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh, blocks);
+    quantize_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+        static_cast<const uint4*>(a.x), a.cos, a.sin, static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh);
   else
-    quantize_unrotated_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(a.x), static_cast<uint2*>(a.codes),
-                                                        a.scale, a.N, blocks_per_bh, blocks);
+    quantize_unrotated_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+        static_cast<const uint4*>(a.x), static_cast<uint2*>(a.codes), a.scale, a.N, blocks_per_bh);
   return cudaGetLastError();
 }
 

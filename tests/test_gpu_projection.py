@@ -123,8 +123,15 @@ def _check_projection(B, N, C, H, seed, rope=True, bias=True, with_bf16=True, at
 
 
 def test_projection_small_ragged():
-    # N not a multiple of the 128-token tile or of the 64-token block; C not a multiple of 64
+    # one-CTA tiles (H = 2); N not a multiple of the 128-token tile or of the 64-token block; C not a
+    # multiple of 64
     _check_projection(B=2, N=300, C=200, H=2, seed=1)
+
+
+def test_projection_pair_tiles_small_ragged():
+    # H a multiple of 4: CTA pairs of 256 tokens x 512 features; the second CTA of the last pair
+    # holds tokens past N
+    _check_projection(B=2, N=300, C=200, H=4, seed=4)
 
 
 def test_projection_without_rope_or_bias():
