@@ -163,7 +163,8 @@ def measured_hbm():
 # The translation unit of each profiled kernel; its counters stay valid while
 # that file and the shared headers are unchanged.
 KERNEL_SOURCES = {"attn_fwd_bf16_kernel": "attn_fwd.cu", "attn_fwd_fp8_kernel": "attn_fwd_fp8.cu",
-                  "merge_kernel": "merge.cu"}
+                  "merge_kernel": "merge.cu", "quantize_kernel": "quant_fp8.cu",
+                  "quantize_unrotated_kernel": "quant_fp8.cu", "qkv_proj_pair_kernel": "qkv_proj.cu"}
 
 
 def profile_traffic(kernel: str):
@@ -224,10 +225,16 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
     s_ptr = stream.cuda_stream
 
     def step(ev=None):
+        if ev is not None:
+            ev[2].record(stream)
         assert lib.dit_attn_quantize_fp8(q.data_ptr(), cos.data_ptr(), sin.data_ptr(), q8.data_ptr(), qs.data_ptr(),
                                          w.B, w.H, w.N, w.D, s_ptr) == 0
+        if ev is not None:
+            ev[3].record(stream)
         assert lib.dit_attn_quantize_fp8(k.data_ptr(), cos.data_ptr(), sin.data_ptr(), k8.data_ptr(), ks.data_ptr(),
                                          w.B, w.H, w.N, w.D, s_ptr) == 0
+        if ev is not None:
+            ev[4].record(stream)
         assert lib.dit_attn_quantize_fp8(v.data_ptr(), None, None, v8.data_ptr(), vs.data_ptr(),
                                          w.B, w.H, w.N, w.D, s_ptr) == 0
         if ev is not None:
@@ -242,7 +249,7 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    kern_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    kern_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(5)) for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -255,7 +262,9 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
     if dit.dit_attn_get_status(stream) != 0:
         raise RuntimeError("device status error in the FP8 timed region")
     max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
-    kern_ms = sum(a.elapsed_time(b) for a, b in kern_ev) / steps
+    kern_ms = sum(e[0].elapsed_time(e[1]) for e in kern_ev) / steps
+    quant_rot_ms = sum(e[2].elapsed_time(e[3]) for e in kern_ev) / steps     # q (rotated)
+    quant_v_ms = sum(e[4].elapsed_time(e[0]) for e in kern_ev) / steps       # v (unrotated)
     peak_bf16, src = measured_peaks()
     # the dense FP8 peak: the measured bf16 peak times the nominal FP8 / BF16 ratio (2)
     peak = 2.0 * peak_bf16
@@ -263,6 +272,22 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
     # (F/2) / (2 P) + (F/2) / P = 0.75 F / P
     peak_mixed = peak_bf16 / 0.75
     achieved = w.flops / (kern_ms * 1e-3) / 1e12
+    # quantiser: 2 B read + 1 B written per element, 4 B per 64-token block scale, and for q, k the
+    # table rows (2 x 64 fp32 per token) once
+    elems = w.B * w.H * w.N * w.D
+    q_bytes = 3 * elems + 4 * w.B * w.H * nb + 512 * w.N
+    v_bytes = 3 * elems + 4 * w.B * w.H * nb
+    hbm = measured_hbm()
+
+    def quant_leg(ms, nbytes, kernel):
+        return {"kernel_ms": ms, "bytes_per_launch": nbytes,
+                "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                             "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "kernel": kernel,
+                             "traffic": profile_traffic(kernel) if w.name == WORKLOAD else None,
+                             "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
+
+    quant = {"rotated": quant_leg(quant_rot_ms, q_bytes, "quantize_kernel"),
+             "unrotated": quant_leg(quant_v_ms, v_bytes, "quantize_unrotated_kernel")}
     return {"value": whole_job_throughput(w.flops, steps, world, max_ms), "unit": UNIT, "steps": steps,
             "ms_per_step": max_ms / steps, "dtype": "e4m3 (q k^T), fp16 (P V)",
             "step": "quantise rotated q, k and v to E4M3 (per 64 tokens) + FP8 attention forward",
@@ -275,7 +300,8 @@ def time_fp8_variant(args, w, lib, q, k, v, cos, sin, out, lse, stream, dev, wor
                          "frac_nominal": achieved / NOMINAL_PEAK_FP8,
                          "note_mixed_peak": {"peak": peak_mixed, "frac": achieved / peak_mixed,
                                              "why": "q k^T on E4M3 at 2x, P V on fp16 at 1x the bf16 rate"},
-                         "kernel_ms": kern_ms}}
+                         "kernel_ms": kern_ms},
+            "quantiser": quant}
 
 
 def time_sparse(args, w, lib, q, k_rot, v_f16, cos, sin, out, lse, stream, dev, dense_ms, density=0.5):
@@ -406,7 +432,9 @@ def time_projection(args, w, lib, cos, sin, stream, dev, C=3072):
             "shape": "x [%d, %d, %d] x w [%d, %d]" % (w.B, w.N, C, 3 * w.H * 128, C),
             "step": "QKV projection GEMM with rotary embedding and E4M3 block quantisation in its epilogue",
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                         "frac": achieved / peak, "kernel": "qkv_proj_fp8_kernel", "traffic": None,
+                         "frac": achieved / peak, "kernel": "qkv_proj_pair_kernel" if w.H % 4 == 0 else "qkv_proj_fp8_kernel",
+                         "traffic": profile_traffic("qkv_proj_pair_kernel") if w.name == WORKLOAD and w.H % 4 == 0
+                         else None,
                          "peak_source": src}}
 
 

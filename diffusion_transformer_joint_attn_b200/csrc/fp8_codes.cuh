@@ -21,22 +21,44 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-// E4M3 code of the correctly rounded fp32 quotient x / scale from
-// r = 1 / scale rounded to nearest (scale and r normal); false if undecided.
-// x * r is within 3 fp32 ulps of that quotient: r and the product are each
-// rounded once, with relative error at most 2^-24.  Rounding to E4M3 is
-// monotonic, so when the fp32 values 8 ulps below and above x * r (the lower
-// magnitude clamped at 0) have one code, the quotient has it too.  They
-// differ when the quotient lies within a few ulps of an E4M3 rounding
-// midpoint (or is not finite); the caller then divides.
-__device__ __forceinline__ bool e4m3_of_quotient(float x, float r, uint32_t& code) {
-  const uint32_t u = __float_as_uint(x * r);
-  const uint32_t mag = u & 0x7FFFFFFFu;
-  const float below = __uint_as_float((u & 0x80000000u) | (max(mag, 8u) - 8u));
-  const float above = __uint_as_float(u + 8u);
-  const uint32_t two = e4m3x2(below, above);
-  code = two & 0xFFu;
-  return ((two ^ (two >> 8)) & 0xFFu) == 0u;
+// E4M3 codes of the correctly rounded fp32 quotients v[e] / scale of 8 values
+// (code e in byte e % 4 of w0 (e < 4) or w1), from r = 1 / scale rounded to
+// nearest (scale and r normal); false if some code is undecided, and then
+// the caller divides.
+//
+// q = RN(v r) is within 3 fp32 ulps of the correctly rounded quotient: r and
+// the product are each rounded once, with relative error at most 2^-24.
+// E4M3 keeps 3 mantissa bits, so in its normal range (|q| >= 2^-6) the
+// rounding midpoints are the fp32 values whose 20 low mantissa bits are
+// 0x80000; rounding is monotonic, so q has the quotient's code unless a
+// midpoint lies within those 3 ulps, i.e. unless q's low bits are within a
+// few units of 0x80000 (tested as: bits 5-19 of q + 8 equal 0x80000, which
+// flags 0x7FFF8 .. 0x80017).  Between 2^-6 and the subnormal codes the
+// spacing changes but no midpoint lies near 2^-6 (the largest subnormal
+// code is 7 x 2^-9); below 2^-6 the midpoints sit elsewhere, so such values
+// (exact zeros included) leave the block undecided, as do ties.
+__device__ __forceinline__ bool e4m3x8_of_quotients(const float* v, float r, uint32_t& w0, uint32_t& w1) {
+  float q[8];
+  float qmin = INFINITY;
+  bool near_midpoint = false;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    q[e] = v[e] * r;
+    qmin = fminf(qmin, fabsf(q[e]));
+    near_midpoint |= ((__float_as_uint(q[e]) + 8u) & 0xFFFE0u) == 0x80000u;
+  }
+  w0 = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
+  w1 = e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16);
+  return !near_midpoint && qmin >= 0.015625f;   // 2^-6
+}
+
+// The same 8 codes through the IEEE division.
+__device__ __forceinline__ void e4m3x8_by_division(const float* v, float scale, uint32_t& w0, uint32_t& w1) {
+  float q[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) q[e] = __fdiv_rn(v[e], scale);
+  w0 = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
+  w1 = e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16);
 }
 
 }  // namespace dit

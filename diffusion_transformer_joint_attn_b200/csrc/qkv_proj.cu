@@ -18,11 +18,12 @@
 // x and sweep the whole weight, which (57 MB at the FLUX width) stays in L2,
 // while x is read from HBM about once.  Warp 0 loads x and w tiles of 64 input channels by TMA into a
 // 4-stage ring, warp 1 issues the MMAs (M = 128, N = 256, K = 16 per
-// instruction) and allocates the 256 tensor-memory columns, warps 2-5 (one
-// thread per token row, lanes by warp & 3) run the epilogue: per head, a
-// first pass over the accumulator for the block maxima, a second for the
-// codes.  The two 64-token blocks of the tile are rows 0-63 (warps 4-5) and
-// 64-127 (warps 2-3).
+// instruction) and allocates the 256 tensor-memory columns, warps 2-9 run
+// the epilogue in two groups of four (one thread per token row in each,
+// lanes by warp & 3), each group taking half of the tile's heads: per head,
+// a first pass over the accumulator for the block maxima, a second for the
+// codes.  The two 64-token blocks of the tile are rows 0-63 (lane quarters
+// 0-1) and 64-127 (quarters 2-3).
 #include <cuda_bf16.h>
 
 #include "fp8_codes.cuh"
@@ -39,9 +40,10 @@ constexpr int kBK = 64;                    // input channels per stage (one 128-
 constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;     // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;     // 32 KB
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
-constexpr int kBarEpi = 1;
+constexpr int kThreads = 320;              // producer, MMA issuer, two epilogue warp groups
+constexpr int kEpiThreads = 128;           // per epilogue warp group
+constexpr int kBarEpi = 1;                 // named barriers 1 and 2, one per epilogue warp group
+constexpr int kMaxTileFeatures = 512;
 
 struct __align__(1024) Smem {
   uint8_t a[kStages][kABytes];
@@ -51,7 +53,8 @@ struct __align__(1024) Smem {
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
-  float block_max[4];                      // per lane quarter of the epilogue warps
+  float block_max[8];                      // per epilogue warp group and lane quarter
+  alignas(16) float bias[kMaxTileFeatures];   // the tile's bias (zeros without one)
 };
 
 struct Params {
@@ -110,13 +113,20 @@ __device__ __forceinline__ void mma_issuer(Smem& sm, const Params& p, uint32_t t
 }
 
 // The 32 accumulator columns at taddr of this thread's row (a warp-collective
-// load: every lane calls it), bias added: y.
-__device__ __forceinline__ void load_y(uint32_t taddr, const Params& p, int o_col, float* y) {
+// load: every lane calls it), plus the bias of those columns (shared memory): y.
+__device__ __forceinline__ void load_y(uint32_t taddr, const float* bias32, float* y) {
   uint32_t u[32];
   tmem_ld32(taddr, u);
   tmem_ld_wait(u);
+  const float4* b4 = reinterpret_cast<const float4*>(bias32);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(u[e]) + (p.bias != nullptr ? __ldg(p.bias + o_col + e) : 0.f);
+  for (int i = 0; i < 8; ++i) {
+    const float4 bb = b4[i];
+    y[4 * i] = __uint_as_float(u[4 * i]) + bb.x;
+    y[4 * i + 1] = __uint_as_float(u[4 * i + 1]) + bb.y;
+    y[4 * i + 2] = __uint_as_float(u[4 * i + 2]) + bb.z;
+    y[4 * i + 3] = __uint_as_float(u[4 * i + 3]) + bb.w;
+  }
 }
 
 // y in place: for q / k each pair rotated with token n's table entries.
@@ -140,37 +150,57 @@ __device__ __forceinline__ void rotate_pairs(const Params& p, int o_col, int n, 
   }
 }
 
-// kHeads heads of 128 accumulator columns each, for the 128 token rows of
-// this CTA starting at token n0; sm supplies acc_full and block_max.
+// The epilogue of kHeads heads (128 accumulator columns each) for the 128
+// token rows of this CTA starting at token n0, by two warp groups (warps 2-5
+// and 6-9, one thread per row in each; warp w reads tensor-memory lanes
+// 32 (w % 4) ...), each taking kHeads / 2 heads; sm supplies acc_full,
+// block_max and the bias slice.  Per head: pass 1 loads y (+ bias), writes
+// the optional bf16 y, rotates q / k pairs, takes the row amax and stores
+// the final values back into the same tensor-memory columns; the block
+// maxima of the two 64-token blocks come from a shuffle and shared-memory
+// reduction over the group; pass 2 reloads the values and encodes them.
 template <int kHeads, typename SmemT>
 __device__ __forceinline__ void epilogue(SmemT& sm, const Params& p, uint32_t tmem, int n0, int o0, int b, int warp,
                                          int lane, const WaitCtx& wc) {
+  constexpr int kGroupHeads = kHeads / 2;
+  const int group = (warp - 2) >> 2;
+  const int gt = ((warp - 2) & 3) * 32 + lane;     // thread within the group
+  const int bar = kBarEpi + group;
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
   const int n = n0 + row;
   const bool valid = n < p.N;
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
   const int nb = (p.N + 63) / 64;
+  // the group's bias columns into shared memory
+  for (int i = gt; i < kGroupHeads * 128; i += kEpiThreads) {
+    const int col = group * kGroupHeads * 128 + i;
+    sm.bias[col] = p.bias != nullptr ? __ldg(p.bias + o0 + col) : 0.f;
+  }
+  named_bar_sync(bar, kEpiThreads);
   const bool ok = warp_wait(&sm.acc_full, 0, wc);
   tc_fence_after();
 #pragma unroll 1
-  for (int head = 0; head < kHeads; ++head) {
+  for (int hh = 0; hh < kGroupHeads; ++hh) {
+    const int head = group * kGroupHeads + hh;
     const int o_head = o0 + head * 128;            // first output feature of the head
     const int which = o_head / (p.H * 128);        // 0 q, 1 k, 2 v
     const int h = (o_head / 128) % p.H;
     const bool rotate = which < 2 && p.cos != nullptr && valid;
     const uint32_t tcol = tmem + lane_base + head * 128;
-    // pass 1: the row's amax, then the block's (and the optional bf16 y)
+    uint8_t* const codes = which == 0 ? p.codes[0] : which == 1 ? p.codes[1] : p.codes[2];
+    float* const scales = which == 0 ? p.scales[0] : which == 1 ? p.scales[1] : p.scales[2];
+    __nv_bfloat16* const y16 = which == 0 ? p.y16[0] : which == 1 ? p.y16[1] : p.y16[2];
+    // pass 1: y, the optional bf16 y, the rotation, the row amax; final values back to tensor memory
     float amax = 0.f;
     if (ok) {
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float r[32];
-        load_y(tcol + q * 32, p, o_head + q * 32, r);
-        if (valid && p.y16[which] != nullptr) {
+        load_y(tcol + q * 32, sm.bias + head * 128 + q * 32, r);
+        if (valid && y16 != nullptr) {
           // unrotated y, rounded to bf16, in the attention layout
-          uint4* dst = reinterpret_cast<uint4*>(p.y16[which] +
-                                                ((static_cast<size_t>(b) * p.H + h) * p.N + n) * 128 + q * 32);
+          uint4* dst = reinterpret_cast<uint4*>(y16 + ((static_cast<size_t>(b) * p.H + h) * p.N + n) * 128 + q * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             dst[e] = make_uint4(pack_bf16x2_rn(r[8 * e], r[8 * e + 1]), pack_bf16x2_rn(r[8 * e + 2], r[8 * e + 3]),
@@ -181,41 +211,36 @@ __device__ __forceinline__ void epilogue(SmemT& sm, const Params& p, uint32_t tm
 #pragma unroll
           for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(r[e]));
         }
+        tmem_st32(tcol + q * 32, reinterpret_cast<const uint32_t*>(r));
       }
+      tmem_st_wait();
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) sm.block_max[quarter] = amax;
-    named_bar_sync(kBarEpi, kEpiThreads);
+    if (lane == 0) sm.block_max[group * 4 + quarter] = amax;
+    named_bar_sync(bar, kEpiThreads);
     const int blk = row >> 6;                      // 64-token block of the tile: quarters 0-1, 2-3
-    const float bmax = fmaxf(sm.block_max[2 * blk], sm.block_max[2 * blk + 1]);
-    named_bar_sync(kBarEpi, kEpiThreads);          // block_max is reused by the next head
+    const float bmax = fmaxf(sm.block_max[group * 4 + 2 * blk], sm.block_max[group * 4 + 2 * blk + 1]);
+    named_bar_sync(bar, kEpiThreads);              // block_max is reused by the next head
     const float scale = bmax == 0.f ? 1.0f : __fdiv_rn(bmax, 448.0f);
-    if ((row & 63) == 0 && valid)
-      p.scales[which][(static_cast<size_t>(b) * p.H + h) * nb + (n0 >> 6) + blk] = scale;
+    if ((row & 63) == 0 && valid) scales[(static_cast<size_t>(b) * p.H + h) * nb + (n0 >> 6) + blk] = scale;
     if (!ok) continue;
     // pass 2: the codes of r / scale (the reciprocal decides when it can);
     // every lane takes part in the warp-collective loads, valid rows store
     const bool via_reciprocal = scale >= 1.17549435e-38f && scale <= 8.50705917e+37f;
     const float rs = __frcp_rn(scale);
-    uint8_t* out = p.codes[which] + ((static_cast<size_t>(b) * p.H + h) * p.N + n) * 128;
+    uint8_t* out = codes + ((static_cast<size_t>(b) * p.H + h) * p.N + n) * 128;
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {
-      float r[32];
-      load_y(tcol + q * 32, p, o_head + q * 32, r);
-      rotate_pairs(p, o_head + q * 32, n, rotate, r);
+      uint32_t u[32];
+      tmem_ld32(tcol + q * 32, u);
+      tmem_ld_wait(u);
+      const float* r = reinterpret_cast<const float*>(u);
       uint32_t word[8];
 #pragma unroll
-      for (int w4 = 0; w4 < 8; ++w4) {
-        uint32_t wd = 0u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x = r[4 * w4 + e];
-          uint32_t code;
-          if (!via_reciprocal || !e4m3_of_quotient(x, rs, code)) code = e4m3x2(__fdiv_rn(x, scale), 0.f) & 0xFFu;
-          wd |= code << (8 * e);
-        }
-        word[w4] = wd;
+      for (int g = 0; g < 4; ++g) {
+        if (!via_reciprocal || !e4m3x8_of_quotients(r + 8 * g, rs, word[2 * g], word[2 * g + 1]))
+          e4m3x8_by_division(r + 8 * g, scale, word[2 * g], word[2 * g + 1]);
       }
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(out + q * 32);
@@ -291,7 +316,8 @@ struct __align__(1024) PairSmem {
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
-  float block_max[4];
+  float block_max[8];
+  alignas(16) float bias[kMaxTileFeatures];
 };
 
 __device__ __forceinline__ uint32_t cl_addr(const void* p, uint32_t rank) { return mapa_shared(smem_u32(p), rank); }

@@ -5,10 +5,11 @@
 // entries (x c - y s with both products exact, one rounding) and rounded to
 // fp32.  The block's scale is amax / 448 in fp32 (1 for an all-zero block);
 // each element becomes the E4M3 code of the fp32 quotient x / scale, rounded
-// to nearest even and saturated to +-448.  The quotient comes from one
+// to nearest even and saturated to +-448.  The quotients come from one
 // multiplication by the block's reciprocal scale whenever that decides the
-// code (e4m3_of_quotient); the IEEE division runs only for quotients within
-// a few ulps of an E4M3 rounding midpoint.
+// codes (e4m3x8_of_quotients, 8 at a time); the IEEE division runs only for
+// the 8 values of a chunk with a quotient near an E4M3 rounding midpoint or
+// below 2^-6.
 #include <cuda_fp8.h>
 
 #include "fp8_codes.cuh"
@@ -22,22 +23,15 @@ constexpr int kThreads = 256;
 constexpr int kChunks = kBlockTokens * 128 / 8;         // 8 channels per chunk
 constexpr int kPerThread = kChunks / kThreads;          // 4
 
-// Element e (0..7) of a chunk held as fp32 values (rotated) or as the raw
-// bf16 words (unrotated: half the registers, so more CTAs stay resident).
-template <bool kRotate>
-struct Chunk;
-template <>
-struct Chunk<true> {
-  float v[8];
-  __device__ __forceinline__ float get(int e) const { return v[e]; }
-};
-template <>
-struct Chunk<false> {
-  uint32_t w[4];
-  __device__ __forceinline__ float get(int e) const {
-    return (e & 1) ? __uint_as_float(w[e >> 1] & 0xFFFF0000u) : __uint_as_float(w[e >> 1] << 16);
-  }
-};
+// 16-byte streaming load: not kept in L1, and L2 fetches the 256-byte
+// sector group around it (the neighbouring threads' chunks).
+__device__ __forceinline__ uint4 ld_stream16(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
 
 template <bool kRotate>
 __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, const float* __restrict__ tc,
@@ -47,7 +41,7 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
   const int bh = blockIdx.x / blocks_per_bh;
   const int blk = blockIdx.x % blocks_per_bh;
   const int n0 = blk * kBlockTokens;
-  Chunk<kRotate> ch[kPerThread];
+  float v[kPerThread][8];               // the thread's chunks as fp32 (rotated for q, k)
   float amax = 0.f;
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
@@ -56,7 +50,7 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
     const int n = n0 + r;
     if (n < N) {
       const long long idx = (static_cast<long long>(bh) * N + n) * 16 + (c & 15);
-      const uint4 w = __ldg(x + idx);
+      const uint4 w = ld_stream16(x + idx);
       if constexpr (kRotate) {
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
         // the four pairs of this chunk: table entries n * 64 + (c & 15) * 4 + 0..3
@@ -66,14 +60,19 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float a = __uint_as_float(ww[e] << 16), b = __uint_as_float(ww[e] & 0xFFFF0000u);
-          ch[u].v[2 * e] = rot_f64(a, cs[e], b, -sn[e]);
-          ch[u].v[2 * e + 1] = rot_f64(a, sn[e], b, cs[e]);
+          v[u][2 * e] = rot_f64(a, cs[e], b, -sn[e]);
+          v[u][2 * e + 1] = rot_f64(a, sn[e], b, cs[e]);
         }
       } else {
-        ch[u].w[0] = w.x, ch[u].w[1] = w.y, ch[u].w[2] = w.z, ch[u].w[3] = w.w;
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[u][2 * e] = __uint_as_float(ww[e] << 16);
+          v[u][2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+        }
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(ch[u].get(e)));
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
     }
   }
 #pragma unroll
@@ -93,35 +92,20 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
     const int c = threadIdx.x + u * kThreads;
     const int n = n0 + (c >> 4);
     if (n >= N) continue;
-    uint32_t word[2] = {0u, 0u};
-    uint32_t divide = via_reciprocal ? 0u : 0xFFu;   // elements whose quotient needs the division
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      uint32_t code;
-      if (!e4m3_of_quotient(ch[u].get(e), r, code)) divide |= 1u << e;
-      word[e >> 2] |= code << (8 * (e & 3));
-    }
-    if (divide != 0u) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (divide & (1u << e)) {
-          const uint32_t code = e4m3x2(__fdiv_rn(ch[u].get(e), scale), 0.f) & 0xFFu;
-          word[e >> 2] = (word[e >> 2] & ~(0xFFu << (8 * (e & 3)))) | (code << (8 * (e & 3)));
-        }
-      }
-    }
+    uint32_t word[2];
+    if (!via_reciprocal || !e4m3x8_of_quotients(v[u], r, word[0], word[1]))
+      e4m3x8_by_division(v[u], scale, word[0], word[1]);
     codes[(static_cast<long long>(bh) * N + n) * 16 + (c & 15)] = make_uint2(word[0], word[1]);
   }
 }
 
-// q, k (rotated): 64 registers, 4 CTAs per SM.  v: the raw words take fewer
-// registers, and 5 CTAs per SM keep more loads in flight.
+// 64 registers: 4 CTAs (32 warps, 64 KB of loads in flight) per SM.
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, const float* __restrict__ tc,
                                                             const float* __restrict__ ts, uint2* __restrict__ codes,
                                                             float* __restrict__ scales, int N, int blocks_per_bh) {
   quantize_block<true>(x, tc, ts, codes, scales, N, blocks_per_bh);
 }
-__global__ void __launch_bounds__(kThreads, 5)
+__global__ void __launch_bounds__(kThreads)
     quantize_unrotated_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes, float* __restrict__ scales, int N,
                               int blocks_per_bh) {
   quantize_block<false>(x, nullptr, nullptr, codes, scales, N, blocks_per_bh);
