@@ -173,11 +173,24 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
     }
     const float neg = -m_used * c;
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t pk[32];
-    exp_half<kPolyEvery<kScaled>>(f, kScaled ? c * sc0 : c, neg, pk, sum);
-    tmem_st32(tS, pk);
-    exp_half<kPolyEvery<kScaled>>(f + 64, kScaled ? c * sc1 : c, neg, pk, sum);
-    tmem_st32(tS + 32, pk);
+    uint32_t pk[kSparse ? 16 : 32];
+    if constexpr (kSparse) {
+      // P in four stores of 16 columns: fewer live registers (the block-sparse
+      // instance holds the tile list state as well); the same pairs, the
+      // same order of the sums, the same bits as the dense instance
+      static_assert(16 % kPolyEvery<kScaled> == 0, "the polynomial pairs must repeat every 16 pairs");
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        exp_pairs<16, kPolyEvery<kScaled>>(f + 32 * q, (kScaled && q >= 2) ? c * sc1 : (kScaled ? c * sc0 : c), neg,
+                                           pk, sum);
+        tmem_st16(tS + 16 * q, pk);
+      }
+    } else {
+      exp_half<kPolyEvery<kScaled>>(f, kScaled ? c * sc0 : c, neg, pk, sum);
+      tmem_st32(tS, pk);
+      exp_half<kPolyEvery<kScaled>>(f + 64, kScaled ? c * sc1 : c, neg, pk, sum);
+      tmem_st32(tS + 32, pk);
+    }
     l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     if (rescale) {
       // O_t holds P V up to tile j-1 (that MMA completed before S_t of
