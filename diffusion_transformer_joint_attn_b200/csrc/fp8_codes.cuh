@@ -31,25 +31,27 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 // E4M3 keeps 3 mantissa bits, so in its normal range (|q| >= 2^-6) the
 // rounding midpoints are the fp32 values whose 20 low mantissa bits are
 // 0x80000; rounding is monotonic, so q has the quotient's code unless a
-// midpoint lies within those 3 ulps, i.e. unless q's low bits are within a
-// few units of 0x80000 (tested as: bits 5-19 of q + 8 equal 0x80000, which
-// flags 0x7FFF8 .. 0x80017).  Between 2^-6 and the subnormal codes the
-// spacing changes but no midpoint lies near 2^-6 (the largest subnormal
-// code is 7 x 2^-9); below 2^-6 the midpoints sit elsewhere, so such values
-// (exact zeros included) leave the block undecided, as do ties.
+// midpoint lies within those 3 ulps.  Decided: no q whose low 20 bits lie in
+// 0x7FFF8 .. 0x80008 (within 8 units of the midpoint; their unsigned
+// distance below 0x7FFF8 wraps above 16), and every q either an exact zero
+// (its code is the quotient's, 0) or at least 2^-6 in magnitude.  Between
+// 2^-6 and the subnormal codes the spacing changes but no midpoint lies near
+// 2^-6 (the largest subnormal code is 7 x 2^-9); below 2^-6 the midpoints sit
+// elsewhere, so such values leave the 8 undecided, as do ties.  Both tests
+// are running unsigned minima over the 8 values.
 __device__ __forceinline__ bool e4m3x8_of_quotients(const float* v, float r, uint32_t& w0, uint32_t& w1) {
   float q[8];
-  float qmin = INFINITY;
-  bool near_midpoint = false;
+  uint32_t mag_min = 0xFFFFFFFFu, dist_min = 0xFFFFFFFFu;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     q[e] = v[e] * r;
-    qmin = fminf(qmin, fabsf(q[e]));
-    near_midpoint |= ((__float_as_uint(q[e]) + 8u) & 0xFFFE0u) == 0x80000u;
+    const uint32_t u = __float_as_uint(q[e]);
+    mag_min = min(mag_min, (u & 0x7FFFFFFFu) - 1u);   // an exact zero wraps to the top
+    dist_min = min(dist_min, (u & 0xFFFFFu) - 0x7FFF8u);
   }
   w0 = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
   w1 = e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16);
-  return !near_midpoint && qmin >= 0.015625f;   // 2^-6
+  return mag_min >= 0x3C800000u - 1u && dist_min > 16u;   // 0x3C800000: 2^-6
 }
 
 // The same 8 codes through the IEEE division.

@@ -9,7 +9,7 @@
 // multiplication by the block's reciprocal scale whenever that decides the
 // codes (e4m3x8_of_quotients, 8 at a time); the IEEE division runs only for
 // the 8 values of a chunk with a quotient near an E4M3 rounding midpoint or
-// below 2^-6.
+// nonzero below 2^-6.
 #include <cuda_fp8.h>
 
 #include "fp8_codes.cuh"
