@@ -46,13 +46,11 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
     const int c = threadIdx.x + u * kThreads;
-    const int r = c >> 4;                      // 16 chunks per token row
-    const int n = n0 + r;
+    const int n = n0 + (c >> 4);               // 16 chunks per token row
     if (n < N) {
-      const long long idx = (static_cast<long long>(bh) * N + n) * 16 + (c & 15);
-      const uint4 w = ld_stream16(x + idx);
+      const uint4 w = ld_stream16(x + (static_cast<long long>(bh) * N + n) * 16 + (c & 15));
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
       if constexpr (kRotate) {
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
         // the four pairs of this chunk: table entries n * 64 + (c & 15) * 4 + 0..3
         const float4 c4 = __ldg(reinterpret_cast<const float4*>(tc) + n * 16 + (c & 15));
         const float4 s4 = __ldg(reinterpret_cast<const float4*>(ts) + n * 16 + (c & 15));
@@ -64,7 +62,6 @@ __device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, cons
           v[u][2 * e + 1] = rot_f64(a, sn[e], b, cs[e]);
         }
       } else {
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           v[u][2 * e] = __uint_as_float(ww[e] << 16);
