@@ -766,7 +766,10 @@ def run_reference(args):
                        step="fp64 oracle: rotary embedding and exact attention of %d sampled query rows" % R),
         "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": threads,
                          "sample": "fp64 numpy oracle: per step the first %d query rows of one head (heads in turn)"
-                                   % R},
+                                   % R,
+                         "extrapolated_full_s": total / args.steps * (w.B * w.H * w.N) / R,
+                         "extrapolated_note": "extrapolated: step time x B*H*N / rows per step; an upper bound, "
+                                              "since each step also pays the head's table and key rotation once"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -781,7 +784,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=W.ORDER, default=WORKLOAD,
                     help="the bench line is the default workload; others serve profiling")
     ap.add_argument("--oracle-rows-per-head", type=int, default=2048)
-    ap.add_argument("--reference-rows", type=int, default=64)
+    ap.add_argument("--reference-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
