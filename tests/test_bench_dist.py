@@ -71,3 +71,9 @@ def test_reference_arm_prints_on_rank_zero_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    # the full-workload time extrapolated from the step time (an upper bound: each step also pays
+    # the head's table and key rotation once): step time x B*H*N / rows per step
+    w = bench.W.WORKLOADS[bench.WORKLOAD]
+    expect = line["ms_per_step"] / 1e3 * w.B * w.H * w.N / 8
+    assert abs(line["cpu_baseline"]["extrapolated_full_s"] - expect) <= 1e-9 * expect
+    assert "extrapolated" in line["cpu_baseline"]["extrapolated_note"]
