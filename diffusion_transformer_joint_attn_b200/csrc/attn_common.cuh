@@ -58,6 +58,19 @@ __device__ __forceinline__ float max64(const float* f) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
+// Max of exactly the 128 values f[0..127] (4 chains of 3-input max).
+__device__ __forceinline__ float max128(const float* f) {
+  float m[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) m[u] = fmaxf(f[2 * u], f[2 * u + 1]);
+#pragma unroll
+  for (int i = 8; i < 128; i += 8) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m[u] = fmax3(m[u], f[i + 2 * u], f[i + 2 * u + 1]);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
 // P for 2 kPairs consecutive logits of the row: 2^(s c - m c) rounded to
 // fp16, packed in pairs into pk[kPairs]; adds the rounded values to sum[4].
 template <int kPairs, int kPoly>
@@ -151,15 +164,14 @@ __device__ __forceinline__ void softmax_slot(const SoftmaxIo& io, uint32_t tmem,
     uint32_t s[128];
 #pragma unroll
     for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, s + q * 32);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld_wait(s + q * 32);
+    tmem_ld_wait128(s);
     float* f = reinterpret_cast<float*>(s);
     if (tail_step && last_valid < kTile) {            // keys past N in the last tile
 #pragma unroll
       for (int e = 0; e < 128; ++e)
         if (e >= last_valid) f[e] = -INFINITY;
     }
-    const float mx = kScaled ? fmaxf(max64(f) * sc0, max64(f + 64) * sc1) : fmaxf(max64(f), max64(f + 64));
+    const float mx = kScaled ? fmaxf(max64(f) * sc0, max64(f + 64) * sc1) : max128(f);
     float alpha = 1.0f;
     bool rescale = false;
     if (i == 0) {

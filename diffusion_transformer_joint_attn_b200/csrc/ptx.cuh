@@ -336,6 +336,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
 __device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" : DIT_INOUT32(r)::"memory");
 }
+// One wait for four 32-column loads into r[0..127].
+__device__ __forceinline__ void tmem_ld_wait128(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : DIT_INOUT32(r), DIT_INOUT32((r + 32)), DIT_INOUT32((r + 64)), DIT_INOUT32((r + 96))::"memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
